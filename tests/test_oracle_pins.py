@@ -1,0 +1,333 @@
+"""Pins for the CPU oracle: each check holds it to something other than itself.
+
+* hand-worked rows (tests/golden/hand_worked.txt, derived on paper);
+* special multipliers that reduce the hash to a plain token shift;
+* brute force over every token string of length <= 5 over {EOS, 1, 2, 3}
+  and every packing, against a restatement that walks the segment
+  explicitly and wraps Python big integers modulo 2^64;
+* invariants: rows inside their head's range, head ranges disjoint, the
+  n-gram after an EOS hashes as at a sequence start, packing position does
+  not matter;
+* the gather against torch.nn.functional.embedding (same definition, library);
+* the gradient against torch.index_add_ in fp64 (integer-valued gradients are
+  exact in any order), the per-row-sum invariant, and closed-form values that
+  only the adopted chunked order (chunks of 32, left folds from the first
+  element, one final add) produces.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from conftest import read_golden_blocks
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+M64 = 1 << 64
+
+
+# ---------------------------------------------------------------------------
+# hash / rows
+# ---------------------------------------------------------------------------
+
+def test_hand_worked_cases():
+    cases, _ = read_golden_blocks("hand_worked.txt")
+    assert len(cases) == 6
+    for c in cases:
+        got = oracle.rows(c["tokens"], c["cu_seqlens"], c["ngram_size"][0], c["heads_per_ngram"][0],
+                          c["eos"][0], c["mults"], c["primes"], c["offsets"])
+        assert got.reshape(-1).tolist() == c["rows"], c["name"]
+
+
+def _ref_rows_bigint(tokens, cu, n, G, eos, mults, primes, offsets):
+    """Independent restatement: for each token, walk back inside its own
+    segment collecting at most n-1 earlier tokens, stopping at an EOS; hash
+    with unbounded integers, wrap to signed 64 bits, floor remainder."""
+    H = (n - 1) * G
+    T = len(tokens)
+    out = np.zeros((T, H), dtype=np.int64)
+    for s in range(len(cu) - 1):
+        seg = tokens[cu[s]:cu[s + 1]]
+        for loc in range(len(seg)):
+            history = []
+            back = loc - 1
+            while back >= 0 and len(history) < n - 1 and seg[back] != eos:
+                history.append(int(seg[back]))
+                back -= 1
+            ctx = [int(seg[loc])] + history + [0] * (n - 1 - len(history))
+            for m in range(2, n + 1):
+                h = sum(ctx[k] * int(mults[k]) for k in range(m)) % M64
+                if h >= 1 << 63:
+                    h -= M64
+                for g in range(G):
+                    j = (m - 2) * G + g
+                    out[cu[s] + loc, j] = int(offsets[j]) + h % int(primes[j])
+    return out
+
+
+def _compositions(L):
+    """All ways to split L tokens into >= 1 consecutive segments, plus one
+    packing with empty segments at both ends and in the middle."""
+    outs = []
+    for cuts in itertools.product([0, 1], repeat=max(L - 1, 0)):
+        cu = [0] + [i + 1 for i, c in enumerate(cuts) if c] + [L]
+        outs.append(cu)
+    half = L // 2
+    outs.append([0, 0, half, half, L, L])
+    return outs
+
+
+@pytest.mark.parametrize("n", [2, 3, 4])
+@pytest.mark.parametrize("mult_kind", ["small", "extreme", "random"])
+def test_brute_force_all_short_strings(n, mult_kind):
+    rng = np.random.default_rng(1000 + n)
+    if mult_kind == "small":
+        mults = [1, 7, 49, 343][:n]
+    elif mult_kind == "extreme":
+        mults = [2 ** 63 - 1, -(2 ** 63), -1, 2 ** 62 + 3][:n]
+    else:
+        mults = synth.signed_mults(n, rng).tolist()
+    G = 2
+    primes = [5, 7, 11, 13, 17, 19][: (n - 1) * G]
+    offsets = synth.exclusive_prefix(primes)
+    eos = 0
+    # pack every case as its own run of sequences in one large packed batch
+    all_tok, all_cu = [], [0]
+    for L in range(1, 6):
+        for s in itertools.product(range(4), repeat=L):
+            for cu in _compositions(L):
+                base = len(all_tok)
+                all_tok.extend(s)
+                all_cu.extend(base + c for c in cu[1:])
+    tok = np.asarray(all_tok, np.int64)
+    cu = np.asarray(all_cu, np.int32)
+    got = oracle.rows(tok, cu, n, G, eos, mults, primes, offsets)
+    ref = _ref_rows_bigint(all_tok, all_cu, n, G, eos, mults, primes, offsets)
+    np.testing.assert_array_equal(got, ref)
+
+
+def _shift_within_segments(tok, cu, k, eos):
+    """Token k positions back, or 0 where that position is before the segment
+    start or an EOS lies in between (numpy shift and masks)."""
+    T = len(tok)
+    seg_start = np.repeat(cu[:-1], np.diff(cu))
+    out = np.zeros(T, np.int64)
+    ok = np.arange(T) - k >= seg_start
+    for d in range(1, k + 1):
+        prev = np.concatenate([np.full(d, -1, np.int64), tok[:-d]]) if d < T else np.full(T, -1, np.int64)
+        ok &= prev != eos
+    src = np.arange(T) - k
+    out[ok] = tok[src[ok]]
+    return out
+
+
+@pytest.mark.parametrize("which", [0, 1, 2, 3])
+def test_shift_only_multipliers(which):
+    """A multiplier vector with a single 1 at slot k makes every order-m head
+    (m > k) a plain remainder of the token k back (or of 0)."""
+    w = synth.tiny(seed=3)
+    n = 4
+    G = 2
+    mults = [0] * n
+    mults[which] = 1
+    primes = synth.consecutive_primes(1009, (n - 1) * G)
+    offsets = synth.exclusive_prefix(primes)
+    got = oracle.rows(w.tokens, w.cu_seqlens, n, G, w.eos_id, mults, primes, offsets)
+    shifted = _shift_within_segments(w.tokens, w.cu_seqlens.astype(np.int64), which, w.eos_id)
+    for j in range(len(primes)):
+        m = 2 + j // G
+        expect = offsets[j] + (np.mod(shifted, primes[j]) if which < m else 0)
+        np.testing.assert_array_equal(got[:, j], expect)
+
+
+def test_rows_in_head_ranges_and_ranges_disjoint():
+    for w in (synth.tiny(0), synth.tiny(5)):
+        r = oracle.rows(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults,
+                        w.primes, w.offsets)
+        lo, hi = w.offsets, w.offsets + w.primes
+        assert np.all(r >= lo[None, :]) and np.all(r < hi[None, :])
+        order = np.argsort(lo)
+        assert np.all(hi[order][:-1] <= lo[order][1:])
+
+
+def test_eos_reset_equals_sequence_start():
+    rng = np.random.default_rng(7)
+    mults = synth.signed_mults(4, rng)
+    primes = synth.consecutive_primes(100_003, 6)
+    offsets = synth.exclusive_prefix(primes)
+    body = rng.integers(1, 1000, 9)
+    with_eos = np.concatenate([[11, 12, 13, 0], body])  # EOS at position 3
+    a = oracle.rows(with_eos, [0, len(with_eos)], 4, 2, 0, mults, primes, offsets)
+    b = oracle.rows(body, [0, len(body)], 4, 2, 0, mults, primes, offsets)
+    np.testing.assert_array_equal(a[4:], b)
+    # the EOS's own n-gram still sees its predecessors
+    c = oracle.rows(with_eos[:4], [0, 4], 4, 2, 0, mults, primes, offsets)
+    np.testing.assert_array_equal(a[:4], c)
+
+
+def test_packing_position_invariance():
+    rng = np.random.default_rng(11)
+    mults = synth.signed_mults(3, rng)
+    primes = synth.consecutive_primes(7919, 4)
+    offsets = synth.exclusive_prefix(primes)
+    seqs = [rng.integers(0, 30, L) for L in (17, 1, 40, 0, 23)]
+    packed = np.concatenate(seqs)
+    cu = synth.cu_seqlens_from_lengths([len(s) for s in seqs])
+    full = oracle.rows(packed, cu, 3, 2, 0, mults, primes, offsets)
+    for s, (a, b) in zip(seqs, zip(cu[:-1], cu[1:])):
+        alone = oracle.rows(s, [0, len(s)], 3, 2, 0, mults, primes, offsets)
+        np.testing.assert_array_equal(full[a:b], alone)
+
+
+def test_malformed_cu_seqlens_rejected():
+    with pytest.raises(ValueError):
+        oracle.rows([1, 2, 3], [0, 2], 2, 1, 0, [1, 1], [7], [0])
+    with pytest.raises(ValueError):
+        oracle.rows([1, 2, 3], [0, 2, 1, 3], 2, 1, 0, [1, 1], [7], [0])
+
+
+def test_production_constants():
+    _, g = read_golden_blocks("production_constants.txt")
+    primes = g["primes_prefix"]
+    # the printed offsets are the exclusive prefix sums of the printed primes
+    assert synth.exclusive_prefix(primes) == g["offsets_prefix"]
+    assert str(g["offsets_prefix"][-1] + primes[-1]).startswith(str(g["offset_9_leading_digits"][0]))
+    # the printed primes are the consecutive primes from 2e7 on
+    assert synth.consecutive_primes(20_000_000, 8) == primes
+    # all 16 heads (ngram 3, 8 per order): their sum, padded to a multiple of 128,
+    # is the printed padded row count
+    all16 = synth.consecutive_primes(20_000_000, 16)
+    total = sum(all16)
+    assert (total + 127) // 128 * 128 == g["padded_rows"][0]
+    # rows of a random stream under the production constants stay in range
+    rng = np.random.default_rng(0)
+    tok = rng.integers(0, 248_320, 3000)
+    tok[rng.random(3000) < 0.01] = g["eos_token_id"][0]
+    offs = synth.exclusive_prefix(all16)
+    r = oracle.rows(tok, [0, 1000, 3000], 3, 8, g["eos_token_id"][0], g["multipliers"], all16, offs)
+    assert r.min() >= 0 and r.max() < total
+    np.testing.assert_array_equal(r, _ref_rows_bigint(tok.tolist(), [0, 1000, 3000], 3, 8,
+                                                      g["eos_token_id"][0], g["multipliers"], all16, offs))
+
+
+def test_multithreaded_rows_match():
+    w = synth.single_layer_bf16(0, total=8192)
+    a = oracle.rows(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
+                    w.offsets)
+    b = oracle.rows(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
+                    w.offsets, threads=4)
+    np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# gather
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [np.float32, np.uint16])
+def test_gather_matches_torch_embedding(dtype):
+    rng = np.random.default_rng(5)
+    table = rng.integers(0, 2 ** 15, size=(997, 24)).astype(dtype) if dtype == np.uint16 else \
+        rng.standard_normal((997, 24)).astype(np.float32)
+    rows = rng.integers(0, 997, size=(50, 6))
+    got = oracle.gather(rows, table)
+    t = torch.from_numpy(table.astype(np.int64) if dtype == np.uint16 else table)
+    ref = torch.nn.functional.embedding(torch.from_numpy(rows), t).numpy().astype(dtype)
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(oracle.gather(rows, table, threads=3), got)
+
+
+def test_gather_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.gather(np.array([0, 5]), np.zeros((5, 4), np.float32))
+    with pytest.raises(ValueError):
+        oracle.gather(np.array([-1]), np.zeros((5, 4), np.float32))
+
+
+# ---------------------------------------------------------------------------
+# gradient
+# ---------------------------------------------------------------------------
+
+def _index_add_fp64(rows, grad_f32, R):
+    D = grad_f32.shape[-1]
+    out = torch.zeros(R, D, dtype=torch.float64)
+    out.index_add_(0, torch.from_numpy(rows.reshape(-1)), torch.from_numpy(grad_f32.reshape(-1, D)).double())
+    return out.numpy()
+
+
+def test_grad_integer_values_exact():
+    rng = np.random.default_rng(9)
+    R, D, N = 300, 16, 5000
+    rows = rng.integers(0, R, N)
+    rows[:700] = 17  # a heavy row spanning many chunks
+    grad = rng.integers(-50, 51, size=(N, D)).astype(np.float32)
+    tg = oracle.grad_apply(rows, grad, np.zeros((R, D), np.float32))
+    np.testing.assert_array_equal(tg.astype(np.float64), _index_add_fp64(rows, grad, R))
+    # bf16 storage of the same small integers is exact too
+    gb = synth.f32_to_bf16_bits(grad)
+    tb = oracle.grad_apply(rows, gb, np.zeros((R, D), np.float32))
+    np.testing.assert_array_equal(tb, tg)
+
+
+def test_grad_random_close_to_fp64_and_row_sum_invariant():
+    w = synth.tiny(0)
+    r = oracle.rows(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
+                    w.offsets)
+    grad = synth.dense_values(w.grad_seed, r.size * w.head_dim, 1.0, synth.DTYPE_F32).reshape(-1, w.head_dim)
+    tg = oracle.grad_apply(r, grad, np.zeros((w.num_rows, w.head_dim), np.float32))
+    ref = _index_add_fp64(r, grad, w.num_rows)
+    np.testing.assert_allclose(tg, ref, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(tg.astype(np.float64).sum(0), grad.astype(np.float64).sum(0), rtol=1e-5, atol=1e-4)
+    uniq, sums = oracle.grad_sums(r, grad)
+    np.testing.assert_array_equal(uniq, np.unique(r))
+    np.testing.assert_array_equal(sums, tg[uniq])
+    u2, s2 = oracle.grad_sums(r, grad, threads=3)
+    np.testing.assert_array_equal(u2, uniq)
+    np.testing.assert_array_equal(s2, sums)
+
+
+def _single_row_grad(values, D=2):
+    N = len(values)
+    rows = np.full(N, 3, np.int64)
+    grad = np.repeat(np.asarray(values, np.float32)[:, None], D, axis=1)
+    return rows, grad
+
+
+def test_grad_chunk_of_32_closed_form():
+    """2^24 followed by 39 ones on one row.  fp32 spacing at 2^24 is 2, so a
+    single left fold loses every 1 (2^24); chunks of 32 give 2^24 (31 ones
+    lost) + 8 = 16777224; chunks of 16 would give 16777240, a pairwise tree
+    16777256."""
+    rows, grad = _single_row_grad([2.0 ** 24] + [1.0] * 39)
+    tg = oracle.grad_apply(rows, grad, np.zeros((5, 2), np.float32))
+    assert tg[3, 0] == np.float32(16777224.0)
+
+
+def test_grad_ascending_index_order_closed_form():
+    """Same multiset in the reverse index order: chunk 0 = 32 ones = 32,
+    chunk 1 = 7 ones then 2^24 = 16777223 -> 16777224 (tie to even), sum
+    16777256: the order of hits inside a row is ascending flat index."""
+    rows, grad = _single_row_grad([1.0] * 39 + [2.0 ** 24])
+    tg = oracle.grad_apply(rows, grad, np.zeros((5, 2), np.float32))
+    assert tg[3, 0] == np.float32(16777256.0)
+
+
+def test_grad_single_final_add_and_negative_zero():
+    # the row sum is formed first and added once: 2^24 + (1 + 1) = 16777218,
+    # while adding the hits into the row one by one would leave 2^24
+    rows, grad = _single_row_grad([1.0, 1.0])
+    tg = np.full((5, 2), 2.0 ** 24, np.float32)
+    oracle.grad_apply(rows, grad, tg)
+    assert tg[3, 0] == np.float32(16777218.0) and tg[0, 0] == np.float32(2.0 ** 24)
+    # folds start from the first element, not from +0: -0 + -0 stays -0
+    rows, grad = _single_row_grad([-0.0])
+    tg = np.full((5, 2), -0.0, np.float32)
+    oracle.grad_apply(rows, grad, tg)
+    assert np.signbit(tg[3, 0])
+
+
+def test_grad_rejects_out_of_range():
+    with pytest.raises(ValueError):
+        oracle.grad_apply(np.array([0, 9]), np.zeros((2, 4), np.float32), np.zeros((5, 4), np.float32))
