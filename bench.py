@@ -1,0 +1,430 @@
+#!/usr/bin/env python3
+"""Throughput of the hashed n-gram (PLE / Engram) lookup on B200.
+
+One step = the whole hot path over one batch of synthetic packed tokens:
+  forward  ple_lookup   (segment/EOS context, order hashes, head rows, row
+                         gather; the rows are saved for the backward)
+  backward ple_grad_scatter (deterministic table gradient of the gather)
+Default workload: 8 packed sequences totalling 32768 tokens (lengths 1k-8k),
+Zipf(1.1) ids over a 151936-id vocabulary, EOS 0.5 %, ngram_size 3, 8 heads
+per order (16 heads), 16 consecutive primes >= 1e6 (16.0M rows), head_dim 64
+bf16 table (2.05 GB); bf16 grad_out N(0,1) into an fp32 table gradient.
+
+Prints ONE JSON line on rank 0 (everything else goes to stderr).
+Multi-GPU: the lookup has no exchange step on one node (one GPU holds the
+whole table), so N GPUs run N independent replicas (weak scaling); ranks
+only meet for a barrier and the max-over-ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "PLE lookup tokens/s and achieved HBM GB/s (fwd gather, bwd scatter) vs 8 TB/s"
+UNIT = "tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+L2_FLUSH_BYTES = 512 << 20   # > 4x the 126 MB L2
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload(name: str, seed: int):
+    import synth
+
+    if name in synth.WORKLOADS:
+        return synth.WORKLOADS[name](seed)
+    if name.startswith("sweep:"):
+        kw = dict(kv.split("=") for kv in name[len("sweep:"):].split(",") if kv)
+        conv = {"tokens": int, "head_dim": int, "ngram_size": int, "heads_per_ngram": int, "table_gb": float,
+                "ids": str}
+        return synth.sweep_point(seed=seed, **{k: conv[k](v) for k, v in kw.items()})
+    raise SystemExit(f"unknown workload {name}")
+
+
+def describe(w):
+    return {"workload": w.name, "tokens": w.num_tokens, "sequences": int(len(w.cu_seqlens) - 1),
+            "ngram_size": w.ngram_size, "heads_per_ngram": w.heads_per_ngram, "heads": w.num_heads,
+            "head_dim": w.head_dim, "table_rows": w.num_rows,
+            "table_dtype": "bf16" if w.table_dtype == 1 else "f32",
+            "table_gb": round(w.table_bytes / 1e9, 3), "grad_dtype": "bf16" if w.grad_dtype == 1 else "f32"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9 or not parts[0].isdigit() or int(parts[0]) != self.gpu:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def traffic_from_profiles(key: str, source_files):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (sha256 prefix recorded beside the number)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    h = hashlib.sha256()
+    for f in source_files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == key and parts[2] == sha:
+            return float(parts[1])
+    return None
+
+
+def cpu_oracle_step(w, table_host, grad_host, threads, tokens_limit=None):
+    """The oracle, as it stands, on the first `tokens_limit` tokens (whole
+    sequences cut at that point): rows, gather, gradient sums."""
+    import oracle
+
+    cu = w.cu_seqlens.astype(np.int64)
+    if tokens_limit is not None and tokens_limit < w.num_tokens:
+        T = tokens_limit
+        cut = cu[cu < T].tolist() + [T]
+        cu = np.asarray(cut, np.int64)
+    else:
+        T = w.num_tokens
+    tok = w.tokens[:T]
+    t0 = time.perf_counter()
+    rows = oracle.rows(tok, cu.astype(np.int32), w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
+                       w.offsets, threads=threads)
+    oracle.gather(rows, table_host, threads=threads)
+    oracle.grad_sums(rows, grad_host[: rows.size], threads=threads)
+    return T, time.perf_counter() - t0
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on bounded samples of the workload."""
+    if rank != 0:
+        return 0
+    import synth
+
+    w = workload(args.workload, args.seed)
+    threads = os.cpu_count() or 1
+    sample = min(w.num_tokens, args.ref_tokens)
+    # host copies of the inputs the sample touches (table rows regenerated on the host)
+    import oracle
+
+    rows_s = oracle.rows(w.tokens[:sample], np.asarray([0] + [c for c in w.cu_seqlens[1:] if c < sample] + [sample],
+                                                         np.int32), w.ngram_size, w.heads_per_ngram, w.eos_id,
+                         w.mults, w.primes, w.offsets)
+    # a full-size host table whose touched rows hold the generated values
+    # (np.zeros pages stay unbacked until written, so untouched rows cost no RAM)
+    table_host = np.zeros((w.num_rows, w.head_dim), np.uint16 if w.table_dtype == 1 else np.float32)
+    uniq = np.unique(rows_s)
+    table_host[uniq] = w.table_rows(uniq)
+    grad_host = synth.dense_values(w.grad_seed, rows_s.size * w.head_dim, w.grad_sigma,
+                                   w.grad_dtype).reshape(rows_s.size, w.head_dim)
+    for _ in range(args.warmup):
+        cpu_oracle_step(w, table_host, grad_host, threads, sample)
+    times = []
+    for _ in range(args.steps):
+        T, dt = cpu_oracle_step(w, table_host, grad_host, threads, sample)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = T / (ms / 1e3)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f32", "data": "synthetic",
+            "config": describe(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"first {T} of {w.num_tokens} tokens per step (rows, gather, grad sums)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="single_layer_bf16")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--fwd-only", action="store_true", help="time the lookup alone (workloads marked fwd only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+
+    import hashed_gram_embedding_ple_b200 as ple
+    import synth
+    from synth import gpu as sgpu
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = workload(args.workload, args.seed + rank)  # each replica its own batch
+    plan = ple.Plan.from_workload(w)
+    T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
+    tdt = torch.bfloat16 if w.table_dtype == 1 else torch.float32
+    gdt = torch.bfloat16 if w.grad_dtype == 1 else torch.float32
+    log(f"[rank {rank}] workload {w.name}: T={T} H={H} D={D} rows={w.num_rows} table {w.table_bytes / 1e9:.2f} GB")
+
+    table = torch.empty(w.num_rows, D, dtype=tdt, device=dev)
+    sgpu.fill_(table, w.table_seed, w.table_sigma)
+    tokens = torch.from_numpy(w.tokens).to(dev)
+    cu = torch.from_numpy(w.cu_seqlens).to(dev)
+    out = torch.empty(T, H, D, dtype=tdt, device=dev)
+    rows = torch.empty(T, H, dtype=torch.int64, device=dev)
+    do_bwd = not args.fwd_only
+    if do_bwd:
+        grad = torch.empty(N, D, dtype=gdt, device=dev)
+        sgpu.fill_(grad, w.grad_seed, w.grad_sigma)
+        table_grad = torch.zeros(w.num_rows, D, dtype=torch.float32, device=dev)
+        ws = ple.alloc_workspace(plan, N, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ple.ple_lookup(plan, tokens, cu, table, out=out, rows_out=rows)
+        if do_bwd:
+            ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
+
+    # unique rows for the backward's algorithmic bytes (bookkeeping, untimed)
+    step()
+    torch.cuda.synchronize()
+    U = int(torch.unique(rows).numel())
+    status = ple.ple_status(dev)
+    if status != ple.PLE_OK:
+        raise SystemExit(f"libple async status {status}")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()                      # L2 flush between steps, outside the events
+        ev[k][0].record(stream)
+        ple.ple_lookup(plan, tokens, cu, table, out=out, rows_out=rows)
+        ev[k][1].record(stream)
+        if do_bwd:
+            ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    status = ple.ple_status(dev)
+    if status != ple.PLE_OK:
+        raise SystemExit(f"libple async status {status}")
+
+    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
+    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
+    step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
+    local = torch.tensor([statistics.mean(step_ms), statistics.mean(fwd_ms), statistics.mean(bwd_ms)],
+                         dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(local, op=dist.ReduceOp.MAX)
+    ms_step, ms_fwd, ms_bwd = [float(x) for x in local.tolist()]
+
+    peak, peak_kind = measured_peaks()
+    e_t = 2 if w.table_dtype == 1 else 4
+    e_g = 2 if w.grad_dtype == 1 else 4
+    fwd_bytes = 8 * T + 2 * N * D * e_t + 8 * N
+    bwd_bytes = 8 * N + N * D * e_g + 2 * U * D * 4
+    fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
+    bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9 if do_bwd else None
+
+    # roofline of the dominant call of the step
+    lookup_src = ["hashed_gram_embedding_ple_b200/csrc/lookup.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+    grad_src = ["hashed_gram_embedding_ple_b200/csrc/grad.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+    fwd_roof = {"bound": "hbm", "achieved": fwd_gbs, "peak": peak, "unit": "GB/s", "frac": fwd_gbs / peak,
+                "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": fwd_bytes,
+                "traffic": traffic_from_profiles(f"lookup_{w.name}", lookup_src), "kernel": "lookup_kernel",
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    roofline = fwd_roof
+    bwd_roof = None
+    if do_bwd:
+        bwd_roof = {"bound": "hbm", "achieved": bwd_gbs, "peak": peak, "unit": "GB/s", "frac": bwd_gbs / peak,
+                    "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": bwd_bytes,
+                    "traffic": traffic_from_profiles(f"grad_scatter_{w.name}", grad_src),
+                    "kernel": "ple_grad_scatter (sort + fold kernels)", "unique_rows": U,
+                    "peak_source": f"{peak_kind} hbm_gbs"}
+        if ms_bwd > ms_fwd:
+            roofline = bwd_roof
+
+    passes = math.ceil(max(1, int(w.num_rows).bit_length()) / 8)
+    launches_per_step = 1 + ((3 * passes + 2) if do_bwd else 0)
+    value = world * T / (ms_step * 1e-3)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        h_tok = torch.from_numpy(w.tokens).pin_memory()
+        h_cu = torch.from_numpy(w.cu_seqlens).pin_memory()
+        h_out = torch.empty(T, H, D, dtype=tdt).pin_memory()
+        h_grad = grad.cpu().pin_memory() if do_bwd else None
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d_tok, d_cu = torch.empty_like(tokens), torch.empty_like(cu)
+        d_grad = torch.empty_like(grad) if do_bwd else None
+        times = []
+        for k in range(args.e2e_steps + 2):
+            flush.zero_()
+            e0.record(stream)
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_cu.copy_(h_cu, non_blocking=True)
+            ple.ple_lookup(plan, d_tok, d_cu, table, out=out, rows_out=rows)
+            if do_bwd:
+                d_grad.copy_(h_grad, non_blocking=True)
+                ple.ple_grad_scatter(plan, rows.view(-1), d_grad, table_grad, workspace=ws)
+            h_out.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if k >= 2:
+                times.append(e0.elapsed_time(e1))
+        t_e2e = torch.tensor([statistics.mean(times)], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+        h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
+        e2e = {"value": world * T / (float(t_e2e.item()) * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": N * D * e_t, "ms_per_step": float(t_e2e.item()),
+               "what": "pinned H2D tokens+cu_seqlens+grad_out, ple_lookup, ple_grad_scatter, D2H of the lookup output"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        uniq_rows = torch.unique(rows)
+        table_host = np.zeros((w.num_rows, D), np.uint16 if w.table_dtype == 1 else np.float32)
+        table_host[uniq_rows.cpu().numpy()] = torch_to_np(table.index_select(0, uniq_rows))
+        grad_host = torch_to_np(grad) if do_bwd else np.zeros((N, D), np.float32)
+        tot_t, tot_s, reps = 0, 0.0, 0
+        while tot_s < args.cpu_seconds and reps < 50:
+            tt, dt = cpu_oracle_step(w, table_host, grad_host, threads)
+            tot_t += tt
+            tot_s += dt
+            reps += 1
+        cpu = {"value": tot_t / tot_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{reps} full passes of the workload ({T} tokens each): rows, gather, gradient sums; "
+                         f"std::thread over sequences / hits / rows, {tot_s:.1f} s"}
+        del table_host
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "int64 hash, bf16 copy, f32 grad", "data": "synthetic",
+                "config": dict(describe(w), parallelism=f"replicas{world}",
+                               l2="512 MB buffer written between steps; flush excluded from step events",
+                               step="ple_lookup (rows saved) + ple_grad_scatter" if do_bwd else "ple_lookup"),
+                "fwd": {"ms": ms_fwd, "tokens_per_s": world * T / (ms_fwd * 1e-3), "gb_per_s": fwd_gbs,
+                        "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "frac_of_measured": fwd_gbs / peak},
+                "bwd": None if not do_bwd else {
+                    "ms": ms_bwd, "tokens_per_s": world * T / (ms_bwd * 1e-3), "gb_per_s": bwd_gbs,
+                    "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "frac_of_measured": bwd_gbs / peak},
+                "roofline": roofline, "roofline_fwd": fwd_roof, "roofline_bwd": bwd_roof,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+                "clocks": clocks, "wall_s_timed_region": wall}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def torch_to_np(t):
+    import torch
+
+    c = t.detach().cpu()
+    if c.dtype == torch.bfloat16:
+        return c.view(torch.int16).numpy().view(np.uint16)
+    return c.numpy()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

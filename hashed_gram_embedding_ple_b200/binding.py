@@ -1,0 +1,240 @@
+"""Thin ctypes binding of libple (include/ple.h).
+
+Argument marshalling only: every step of the lookup runs in the library's
+CUDA kernels.  PyTorch supplies device memory (output and workspace tensors
+are allocated here with torch when the caller does not pass them) and the
+current CUDA stream.  There is no fallback: if libple.so is missing or a
+call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from ._build import LIB_PATH
+
+PLE_OK = 0
+PLE_ERR_INVALID_ARG = 1
+PLE_ERR_UNSUPPORTED = 2
+PLE_ERR_ALIGNMENT = 3
+PLE_ERR_WORKSPACE = 4
+PLE_ERR_CUDA = 5
+PLE_ERR_BAD_ROW = 6
+PLE_ERR_BAD_SEQLENS = 7
+
+PLE_F32 = 0
+PLE_BF16 = 1
+
+_DTYPES = {torch.float32: PLE_F32, torch.bfloat16: PLE_BF16}
+
+# every symbol include/ple.h declares
+EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_gather",
+           "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic", "ple_status",
+           "ple_strerror", "ple_last_cuda_error")
+
+
+class PleError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib().ple_strerror(status).decode()
+        if status == PLE_ERR_CUDA:
+            msg += f" (cudaError {_lib().ple_last_cuda_error()})"
+        super().__init__(f"{where}: {msg} [status {status}]")
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("ngram_size", ctypes.c_int32), ("heads_per_ngram", ctypes.c_int32), ("eos_id", ctypes.c_int64),
+                ("mults", ctypes.POINTER(ctypes.c_int64)), ("primes", ctypes.POINTER(ctypes.c_int64)),
+                ("offsets", ctypes.POINTER(ctypes.c_int64)), ("num_rows", ctypes.c_int64),
+                ("head_dim", ctypes.c_int32), ("table_dtype", ctypes.c_int)]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libple is not built ({LIB_PATH}); run __graft_entry__.build() or "
+                              "python -m hashed_gram_embedding_ple_b200._build")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        lib.ple_plan_create.argtypes = [ctypes.POINTER(_Params), ctypes.POINTER(vp)]
+        lib.ple_plan_destroy.argtypes = [vp]
+        lib.ple_plan_destroy.restype = None
+        lib.ple_plan_num_heads.argtypes = [vp]
+        lib.ple_plan_num_heads.restype = i32
+        lib.ple_hash.argtypes = [vp, vp, i64, vp, i32, vp, vp]
+        lib.ple_lookup.argtypes = [vp, vp, i64, vp, i32, vp, vp, vp, vp]
+        lib.ple_gather.argtypes = [vp, vp, i64, vp, vp, vp]
+        lib.ple_grad_scatter_workspace_bytes.argtypes = [vp, i64]
+        lib.ple_grad_scatter_workspace_bytes.restype = sz
+        lib.ple_grad_scatter.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
+        lib.ple_grad_scatter_atomic.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
+        lib.ple_status.argtypes = [vp]
+        lib.ple_strerror.argtypes = [ctypes.c_int]
+        lib.ple_strerror.restype = ctypes.c_char_p
+        lib.ple_last_cuda_error.argtypes = []
+        for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_gather", "ple_grad_scatter",
+                     "ple_grad_scatter_atomic", "ple_status", "ple_last_cuda_error"):
+            getattr(lib, name).restype = ctypes.c_int
+        _LIB = lib
+    return _LIB
+
+
+def lib():
+    """The loaded libple CDLL (raises ImportError if it is not built)."""
+    return _lib()
+
+
+def _check(rc: int, where: str):
+    if rc != PLE_OK:
+        raise PleError(rc, where)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+class Plan:
+    """Hash and table description (ple_params_t) validated by ple_plan_create."""
+
+    def __init__(self, ngram_size, heads_per_ngram, eos_id, mults, primes, offsets, num_rows, head_dim,
+                 table_dtype=torch.bfloat16):
+        H = (ngram_size - 1) * heads_per_ngram
+        self._mults = (ctypes.c_int64 * max(1, len(mults)))(*[int(m) for m in mults])
+        self._primes = (ctypes.c_int64 * max(1, len(primes)))(*[int(p) for p in primes])
+        self._offsets = (ctypes.c_int64 * max(1, len(offsets)))(*[int(o) for o in offsets])
+        if len(mults) != ngram_size or len(primes) != H or len(offsets) != H:
+            raise ValueError("mults must have ngram_size entries; primes and offsets (ngram_size-1)*heads_per_ngram")
+        if table_dtype not in _DTYPES:
+            raise ValueError(f"table dtype must be float32 or bfloat16, not {table_dtype}")
+        p = _Params(ngram_size, heads_per_ngram, int(eos_id), self._mults, self._primes, self._offsets,
+                    int(num_rows), int(head_dim), _DTYPES[table_dtype])
+        handle = ctypes.c_void_p()
+        _check(_lib().ple_plan_create(ctypes.byref(p), ctypes.byref(handle)), "ple_plan_create")
+        self._h = handle
+        self.ngram_size, self.heads_per_ngram, self.num_heads = ngram_size, heads_per_ngram, H
+        self.num_rows, self.head_dim, self.table_dtype = int(num_rows), int(head_dim), table_dtype
+
+    @classmethod
+    def from_workload(cls, w):
+        return cls(w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes, w.offsets, w.num_rows,
+                   w.head_dim, torch.float32 if w.table_dtype == PLE_F32 else torch.bfloat16)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _LIB is not None:
+            _LIB.ple_plan_destroy(h)
+            self._h = None
+
+
+def _as_i64(t, name):
+    if t.dtype != torch.int64 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous int64 CUDA tensor")
+
+
+def _as_i32(t, name):
+    if t.dtype != torch.int32 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+
+
+def ple_hash(plan: Plan, tokens, cu_seqlens, rows=None):
+    """int64 [T, H] global rows of every (token, head)."""
+    _as_i64(tokens, "tokens")
+    _as_i32(cu_seqlens, "cu_seqlens")
+    T = tokens.numel()
+    if rows is None:
+        rows = torch.empty(T, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    _check(_lib().ple_hash(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, _ptr(rows),
+                           _stream(tokens.device)), "ple_hash")
+    return rows
+
+
+def ple_lookup(plan: Plan, tokens, cu_seqlens, table, out=None, rows_out=None, save_rows: bool = False):
+    """Hash fused with the gather: [T, H, D] values in the table dtype.
+    With save_rows (or a rows_out tensor) also returns the [T, H] rows."""
+    _as_i64(tokens, "tokens")
+    _as_i32(cu_seqlens, "cu_seqlens")
+    if table.dtype != plan.table_dtype or not table.is_contiguous() or table.shape[-1] != plan.head_dim:
+        raise ValueError("table must be contiguous [num_rows, head_dim] in the plan's dtype")
+    T = tokens.numel()
+    if out is None:
+        out = torch.empty(T, plan.num_heads, plan.head_dim, dtype=table.dtype, device=table.device)
+    if rows_out is None and save_rows:
+        rows_out = torch.empty(T, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    _check(_lib().ple_lookup(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                             _ptr(table), _ptr(out), _ptr(rows_out), _stream(tokens.device)), "ple_lookup")
+    return (out, rows_out) if rows_out is not None else out
+
+
+def ple_gather(plan: Plan, rows, table, out=None):
+    """out[i] = table[rows[i]] for flat rows; shape rows.shape + [D]."""
+    _as_i64(rows, "rows")
+    if table.dtype != plan.table_dtype or not table.is_contiguous():
+        raise ValueError("table must be contiguous in the plan's dtype")
+    if out is None:
+        out = torch.empty(*rows.shape, plan.head_dim, dtype=table.dtype, device=table.device)
+    _check(_lib().ple_gather(plan.handle, _ptr(rows), rows.numel(), _ptr(table), _ptr(out),
+                             _stream(rows.device)), "ple_gather")
+    return out
+
+
+def workspace_bytes(plan: Plan, num_hits: int) -> int:
+    return int(_lib().ple_grad_scatter_workspace_bytes(plan.handle, int(num_hits)))
+
+
+def alloc_workspace(plan: Plan, num_hits: int, device):
+    n = workspace_bytes(plan, num_hits)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+
+
+def _grad_dtype(g):
+    if g.dtype not in _DTYPES or not g.is_contiguous():
+        raise ValueError("grad_out must be contiguous float32 or bfloat16")
+    return _DTYPES[g.dtype]
+
+
+def ple_grad_scatter(plan: Plan, rows, grad_out, table_grad, workspace=None):
+    """Deterministic table_grad += per-row sums of grad_out (fixed chunked order)."""
+    _as_i64(rows, "rows")
+    gdt = _grad_dtype(grad_out)
+    if table_grad.dtype != torch.float32 or not table_grad.is_contiguous():
+        raise ValueError("table_grad must be contiguous float32")
+    N = rows.numel()
+    if grad_out.numel() != N * plan.head_dim:
+        raise ValueError("grad_out must hold num_hits * head_dim values")
+    if workspace is None:
+        workspace = alloc_workspace(plan, N, rows.device)
+    _check(_lib().ple_grad_scatter(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
+                                   _ptr(workspace), workspace.numel(), _stream(rows.device)), "ple_grad_scatter")
+    return table_grad
+
+
+def ple_grad_scatter_atomic(plan: Plan, rows, grad_out, table_grad):
+    """Non-deterministic fp32 atomic variant (speed reference)."""
+    _as_i64(rows, "rows")
+    gdt = _grad_dtype(grad_out)
+    N = rows.numel()
+    if grad_out.numel() != N * plan.head_dim:
+        raise ValueError("grad_out must hold num_hits * head_dim values")
+    _check(_lib().ple_grad_scatter_atomic(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
+                                          _stream(rows.device)), "ple_grad_scatter_atomic")
+    return table_grad
+
+
+def ple_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the async status."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(_lib().ple_status(_stream(dev)))

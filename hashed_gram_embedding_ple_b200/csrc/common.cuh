@@ -1,0 +1,108 @@
+// Internal definitions shared by the libple translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "ple.h"
+
+namespace ple {
+
+constexpr int kMaxOrder = 8;   // ngram_size limit
+constexpr int kMaxHeads = 64;  // H limit
+
+// Per-head remainder constants.  For a modulus p (2 <= p <= 2^62):
+//   magic = floor((2^64 - 1) / p), wrap = 2^64 mod p.
+// q = mulhi(u, magic) underestimates floor(u / p) by at most 2 (Barrett,
+// "Implementing the RSA public key encryption algorithm on a standard
+// digital signal processor", CRYPTO 1986, with a one-word reciprocal), so
+// u - q*p lies in [0, 3p) and two conditional subtractions finish u mod p.
+struct HeadConst {
+  uint64_t prime;
+  uint64_t magic;
+  uint64_t wrap;
+  int64_t offset;
+};
+
+// Everything a hash kernel needs, passed by value as a kernel parameter.
+struct HashParams {
+  int32_t ngram_size;
+  int32_t heads_per_ngram;
+  int32_t num_heads;
+  int32_t pad_;
+  int64_t eos_id;
+  int64_t mults[kMaxOrder];
+  HeadConst head[kMaxHeads];
+};
+
+// Floor remainder of a signed 64-bit value: ((h % p) + p) % p.
+__device__ __forceinline__ uint64_t floor_mod(int64_t h, const HeadConst& c) {
+  const uint64_t u = static_cast<uint64_t>(h);
+  const uint64_t q = __umul64hi(u, c.magic);
+  uint64_t r = u - q * c.prime;
+  if (r >= c.prime) r -= c.prime;
+  if (r >= c.prime) r -= c.prime;
+  // h < 0: h = u - 2^64, so h mod p = (u mod p - 2^64 mod p) mod p
+  if (h < 0) r = (r >= c.wrap) ? r - c.wrap : r + c.prime - c.wrap;
+  return r;
+}
+
+// 16-byte load that bypasses L1 allocation (rows are touched once per hit).
+__device__ __forceinline__ uint4 ld_nc_na(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// 16-byte streaming store (evict-first: the output is not re-read here).
+__device__ __forceinline__ void st_cs(void* p, const uint4& v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+// Async status bits (bit k-1 for status code k).
+__device__ __forceinline__ void raise_flag(unsigned int* status, ple_status_t code) {
+  atomicOr(status, 1u << (static_cast<int>(code) - 1));
+}
+
+// Index s of the packed sequence holding token t: the last s with
+// cu[s] <= t, searched over cu[0..num_seqs) (clamped to [0, num_seqs-1]).
+__device__ __forceinline__ int32_t find_sequence(const int32_t* __restrict__ cu, int32_t num_seqs,
+                                                 int64_t t) {
+  int32_t lo = 0, hi = num_seqs - 1;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi + 1) >> 1;
+    if (static_cast<int64_t>(__ldg(cu + mid)) <= t)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace ple
+
+// ---------------------------------------------------------------------------
+// Host-side internals (defined in plan.cu)
+// ---------------------------------------------------------------------------
+struct ple_plan {
+  ple::HashParams hp;
+  int64_t num_rows;
+  int32_t head_dim;
+  ple_dtype_t table_dtype;
+  int32_t row_bytes;
+};
+
+namespace ple {
+// Device address of the async status word for the current device.
+unsigned int* status_word(cudaError_t* err);
+// Multiprocessor count of the current device (cached).
+int sm_count();
+// Record a CUDA error for ple_last_cuda_error and return PLE_ERR_CUDA.
+ple_status_t cuda_fail(cudaError_t e);
+// PLE_OK, or cuda_fail of the last launch error.
+ple_status_t check_launch();
+}  // namespace ple

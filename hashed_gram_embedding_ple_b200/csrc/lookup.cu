@@ -1,0 +1,342 @@
+// Forward path: row hashing (_hash_input_ids), the fused hash + row gather
+// (forward of Qwen3_8_FlashNextNGramEmbedding) and the plain row gather
+// (_lookup_ngram_ids), NeMo AutoModel engram API page.
+//
+// The gather is HBM-bound: every hit reads one table row and writes one
+// output row.  A block stages the byte offsets of its hits in shared memory,
+// then streams the rows as flat 16-byte vectors: vector q of the block's
+// output is column (q mod V) of hit (q div V), V = row_bytes / 16, so the
+// stores of a warp are contiguous and each row is read by V consecutive
+// lanes.  UNROLL independent loads are in flight per thread before the
+// matching stores are issued.
+#include "common.cuh"
+
+namespace ple {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kBlock = 256;     // threads per block of the gather kernels
+constexpr int kUnroll = 8;      // 16-byte loads in flight per thread
+constexpr int kHashWarps = 4;   // warps per block of the stand-alone hash
+
+// Block 0 checks cu_seqlens once per launch: cu[0] == 0, cu[S] == T and
+// non-decreasing.  Bad input only raises a flag; all indexing stays in range.
+__device__ void check_seqlens(const int32_t* __restrict__ cu, int32_t num_seqs, int64_t T,
+                              unsigned int* status) {
+  if (blockIdx.x != 0) return;
+  bool bad = false;
+  if (threadIdx.x == 0) bad = (cu[0] != 0) || (static_cast<int64_t>(cu[num_seqs]) != T);
+  for (int32_t s = threadIdx.x; s < num_seqs; s += blockDim.x) bad |= cu[s + 1] < cu[s];
+  if (bad) raise_flag(status, PLE_ERR_BAD_SEQLENS);
+}
+
+// Order hashes h_2..h_n of token t, the token of this lane.  Called by a
+// whole warp; lanes hold consecutive tokens (valid lanes form a prefix).
+// The previous tokens come from lower lanes by shuffle; the first k lanes
+// load the k-token halo before the warp's first token from global memory.
+// Context slot k is kept while position t-k is inside t's packed sequence
+// and no EOS sits in positions t-k .. t-1; otherwise it and every slot
+// beyond it hold the sentinel 0.
+__device__ __forceinline__ void order_hashes(const HashParams& hp, const int64_t* __restrict__ tokens,
+                                             const int32_t* __restrict__ cu, int32_t num_seqs, int64_t t,
+                                             bool valid, int64_t (&hs)[kMaxOrder - 1]) {
+  const int lane = threadIdx.x & 31;
+  const int64_t tok = valid ? tokens[t] : 0;
+  const int64_t seq_start = valid ? static_cast<int64_t>(cu[find_sequence(cu, num_seqs, t)]) : 0;
+  uint64_t h = static_cast<uint64_t>(tok) * static_cast<uint64_t>(hp.mults[0]);
+  bool keep = valid;
+#pragma unroll
+  for (int k = 1; k < kMaxOrder; ++k) {
+    if (k < hp.ngram_size) {
+      int64_t prev = __shfl_up_sync(kFull, tok, k);
+      if (lane < k) prev = (valid && t - k >= 0) ? tokens[t - k] : 0;
+      keep = keep && (t - k >= seq_start) && (prev != hp.eos_id);
+      const int64_t ctx = keep ? prev : 0;
+      h += static_cast<uint64_t>(ctx) * static_cast<uint64_t>(hp.mults[k]);
+      hs[k - 1] = static_cast<int64_t>(h);
+    }
+  }
+}
+
+// rows of the tokens of this lane for every head, head j of order 2 + j/G.
+template <typename Emit>
+__device__ __forceinline__ void rows_of_token(const HashParams& hp, const HeadConst* consts,
+                                              const int64_t (&hs)[kMaxOrder - 1], Emit emit) {
+  const int G = hp.heads_per_ngram;
+#pragma unroll
+  for (int m = 0; m < kMaxOrder - 1; ++m) {
+    if (m < hp.ngram_size - 1) {
+      for (int g = 0; g < G; ++g) {
+        const int j = m * G + g;
+        const HeadConst c = consts[j];
+        emit(j, c.offset + static_cast<int64_t>(floor_mod(hs[m], c)));
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void load_consts(const HashParams& hp, HeadConst* consts) {
+  for (int j = threadIdx.x; j < hp.num_heads; j += blockDim.x) consts[j] = hp.head[j];
+}
+
+// ---------------------------------------------------------------------------
+// Stand-alone hash: one warp per 32 tokens, staged through shared memory so
+// that the int64 [T, H] rows are written with coalesced stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kHashWarps * 32)
+hash_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
+            const int32_t* __restrict__ cu, int32_t num_seqs, int64_t* __restrict__ rows,
+            unsigned int* status) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  HeadConst* consts = reinterpret_cast<HeadConst*>(smem);
+  const int H = hp.num_heads;
+  int64_t* stage = reinterpret_cast<int64_t*>(consts + H) + (threadIdx.x >> 5) * 32 * H;
+  load_consts(hp, consts);
+  check_seqlens(cu, num_seqs, T, status);
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int64_t t_first = (static_cast<int64_t>(blockIdx.x) * kHashWarps + (threadIdx.x >> 5)) * 32;
+  if (t_first >= T) return;
+  const int64_t t = t_first + lane;
+  const bool valid = t < T;
+  int64_t hs[kMaxOrder - 1];
+  order_hashes(hp, tokens, cu, num_seqs, t, valid, hs);
+  rows_of_token(hp, consts, hs, [&](int j, int64_t row) { stage[lane * H + j] = row; });
+  __syncwarp();
+  const int n = static_cast<int>(min(static_cast<int64_t>(32), T - t_first)) * H;
+  int64_t* dst = rows + t_first * H;
+  for (int q = lane; q < n; q += 32) dst[q] = stage[q];
+}
+
+// ---------------------------------------------------------------------------
+// Row streaming shared by the fused lookup and the gather.
+// ---------------------------------------------------------------------------
+template <int VL>
+__device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ table,
+                                          const int64_t* __restrict__ rowoff, int nhits, int v_rt,
+                                          unsigned char* __restrict__ out) {
+  const int V = VL >= 0 ? (1 << VL) : v_rt;
+  const int total = nhits * V;
+  for (int base = threadIdx.x; base < total; base += kBlock * kUnroll) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int q = base + u * kBlock;
+      if (q < total) {
+        const int hit = VL >= 0 ? (q >> VL) : q / V;
+        const int col = q - hit * V;
+        const int64_t off = rowoff[hit];
+        v[u] = off >= 0 ? ld_nc_na(table + off + col * 16) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int q = base + u * kBlock;
+      if (q < total) st_cs(out + static_cast<int64_t>(q) * 16, v[u]);
+    }
+  }
+}
+
+// Fused lookup: TT tokens per block.  Warp 0 hashes the tile's tokens, all
+// threads turn the order hashes into rows (one remainder per hit), then the
+// block streams the tile's TT*H rows.
+template <int TT, int VL>
+__global__ void __launch_bounds__(kBlock, 4)
+lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
+              const int32_t* __restrict__ cu, int32_t num_seqs, const unsigned char* __restrict__ table,
+              int64_t num_rows, int32_t row_bytes, unsigned char* __restrict__ out,
+              int64_t* __restrict__ rows_out, unsigned int* status) {
+  static_assert(TT <= 32, "one warp hashes the tile");
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int H = hp.num_heads;
+  HeadConst* consts = reinterpret_cast<HeadConst*>(smem);
+  int64_t* hsh = reinterpret_cast<int64_t*>(consts + H);   // [TT][kMaxOrder-1]
+  int64_t* rowoff = hsh + TT * (kMaxOrder - 1);            // [TT*H]
+  load_consts(hp, consts);
+  check_seqlens(cu, num_seqs, T, status);
+
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * TT;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int64_t t = t0 + lane;
+    const bool valid = lane < TT && t < T;
+    int64_t hs[kMaxOrder - 1];
+    order_hashes(hp, tokens, cu, num_seqs, t, valid, hs);
+    if (lane < TT) {
+#pragma unroll
+      for (int m = 0; m < kMaxOrder - 1; ++m) hsh[lane * (kMaxOrder - 1) + m] = hs[m];
+    }
+  }
+  __syncthreads();
+
+  const int ntok = static_cast<int>(min(static_cast<int64_t>(TT), T - t0));
+  const int nhits = ntok * H;
+  const int G = hp.heads_per_ngram;
+  for (int q = threadIdx.x; q < nhits; q += kBlock) {
+    const int tl = q / H;
+    const int j = q - tl * H;
+    const HeadConst c = consts[j];
+    const int64_t row = c.offset + static_cast<int64_t>(floor_mod(hsh[tl * (kMaxOrder - 1) + j / G], c));
+    // always true for a validated plan; kept so that no table read can leave the table
+    rowoff[q] = row < num_rows ? row * row_bytes : -1;
+    if (rows_out != nullptr) rows_out[t0 * H + q] = row;
+  }
+  __syncthreads();
+  copy_hits<VL>(table, rowoff, nhits, row_bytes >> 4, out + t0 * H * row_bytes);
+}
+
+constexpr int kGatherHits = 512;  // hits per block of the plain gather
+
+template <int VL>
+__global__ void __launch_bounds__(kBlock, 4)
+gather_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows,
+              const unsigned char* __restrict__ table, int32_t row_bytes, unsigned char* __restrict__ out,
+              unsigned int* status) {
+  __shared__ int64_t rowoff[kGatherHits];
+  const int64_t h0 = static_cast<int64_t>(blockIdx.x) * kGatherHits;
+  const int nh = static_cast<int>(min(static_cast<int64_t>(kGatherHits), N - h0));
+  bool bad = false;
+  for (int q = threadIdx.x; q < nh; q += kBlock) {
+    const int64_t r = rows[h0 + q];
+    const bool ok = r >= 0 && r < num_rows;
+    bad |= !ok;
+    rowoff[q] = ok ? r * row_bytes : -1;
+  }
+  if (bad) raise_flag(status, PLE_ERR_BAD_ROW);
+  __syncthreads();
+  copy_hits<VL>(table, rowoff, nh, row_bytes >> 4, out + h0 * row_bytes);
+}
+
+int log2_exact(int v) {
+  for (int k = 0; k < 31; ++k)
+    if ((1 << k) == v) return k;
+  return -1;
+}
+
+template <int TT>
+ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                           int32_t S, const void* table, void* out, int64_t* rows_out, unsigned int* status,
+                           cudaStream_t stream) {
+  const int H = plan->hp.num_heads;
+  const size_t smem = H * sizeof(HeadConst) + TT * (kMaxOrder - 1) * sizeof(int64_t) +
+                      static_cast<size_t>(TT) * H * sizeof(int64_t);
+  const dim3 grid(static_cast<unsigned>((T + TT - 1) / TT));
+  const auto* tb = static_cast<const unsigned char*>(table);
+  auto* ob = static_cast<unsigned char*>(out);
+  const int rb = plan->row_bytes;
+  const int64_t R = plan->num_rows;
+#define PLE_LOOKUP_CASE(VL)                                                                           \
+  case VL:                                                                                            \
+    lookup_kernel<TT, VL><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,     \
+                                                          rows_out, status);                                     \
+    break;
+  switch (log2_exact(rb >> 4)) {
+    PLE_LOOKUP_CASE(0)
+    PLE_LOOKUP_CASE(1)
+    PLE_LOOKUP_CASE(2)
+    PLE_LOOKUP_CASE(3)
+    PLE_LOOKUP_CASE(4)
+    PLE_LOOKUP_CASE(5)
+    PLE_LOOKUP_CASE(6)
+    default:
+      lookup_kernel<TT, -1><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
+                                                            rows_out, status);
+  }
+#undef PLE_LOOKUP_CASE
+  return check_launch();
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+ple_status_t check_hash_args(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                             int32_t S) {
+  if (plan == nullptr || T < 0) return PLE_ERR_INVALID_ARG;
+  if (T == 0) return PLE_OK;
+  if (tokens == nullptr || cu == nullptr || S < 1) return PLE_ERR_INVALID_ARG;
+  if (T > (int64_t{1} << 40)) return PLE_ERR_UNSUPPORTED;
+  if (!aligned(tokens, 8) || !aligned(cu, 4)) return PLE_ERR_ALIGNMENT;
+  return PLE_OK;
+}
+
+}  // namespace
+}  // namespace ple
+
+using namespace ple;
+
+extern "C" {
+
+ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                      int32_t S, int64_t* rows, void* stream) {
+  ple_status_t st = check_hash_args(plan, tokens, T, cu, S);
+  if (st != PLE_OK || T == 0) return st;
+  if (rows == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(rows, 8)) return PLE_ERR_ALIGNMENT;
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const int H = plan->hp.num_heads;
+  const size_t smem = H * sizeof(HeadConst) + static_cast<size_t>(kHashWarps) * 32 * H * sizeof(int64_t);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(hash_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  const int64_t warps = (T + 31) / 32;
+  const dim3 grid(static_cast<unsigned>((warps + kHashWarps - 1) / kHashWarps));
+  hash_kernel<<<grid, kHashWarps * 32, smem, static_cast<cudaStream_t>(stream)>>>(plan->hp, tokens, T, cu, S,
+                                                                                   rows, status);
+  return check_launch();
+}
+
+ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                        int32_t S, const void* table, void* out, int64_t* rows_out, void* stream) {
+  ple_status_t st = check_hash_args(plan, tokens, T, cu, S);
+  if (st != PLE_OK || T == 0) return st;
+  if (table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(table, 16) || !aligned(out, 16) || (rows_out != nullptr && !aligned(rows_out, 8)))
+    return PLE_ERR_ALIGNMENT;
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const int64_t tiles32 = (T + 31) / 32;
+  const auto s = static_cast<cudaStream_t>(stream);
+  if (tiles32 >= 8LL * sm_count())
+    return launch_lookup<32>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+  return launch_lookup<16>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+}
+
+ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* table, void* out,
+                        void* stream) {
+  if (plan == nullptr || N < 0) return PLE_ERR_INVALID_ARG;
+  if (N == 0) return PLE_OK;
+  if (rows == nullptr || table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(rows, 8) || !aligned(table, 16) || !aligned(out, 16)) return PLE_ERR_ALIGNMENT;
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const dim3 grid(static_cast<unsigned>((N + kGatherHits - 1) / kGatherHits));
+  const auto s = static_cast<cudaStream_t>(stream);
+  const auto* tb = static_cast<const unsigned char*>(table);
+  auto* ob = static_cast<unsigned char*>(out);
+  const int rb = plan->row_bytes;
+  const int64_t R = plan->num_rows;
+#define PLE_GATHER_CASE(VL)                                                       \
+  case VL:                                                                        \
+    gather_kernel<VL><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);    \
+    break;
+  switch (log2_exact(rb >> 4)) {
+    PLE_GATHER_CASE(0)
+    PLE_GATHER_CASE(1)
+    PLE_GATHER_CASE(2)
+    PLE_GATHER_CASE(3)
+    PLE_GATHER_CASE(4)
+    PLE_GATHER_CASE(5)
+    PLE_GATHER_CASE(6)
+    default:
+      gather_kernel<-1><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
+  }
+#undef PLE_GATHER_CASE
+  return check_launch();
+}
+
+}  // extern "C"

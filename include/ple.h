@@ -1,0 +1,162 @@
+/*
+ * ple.h -- C ABI of libple, a B200 (sm_100a) implementation of the hashed
+ * n-gram ("PLE" / Engram) embedding lookup of Qwen3.8-Flash-Next.
+ *
+ * The operations follow the NeMo AutoModel API page
+ * "nemo_automodel.components.models.qwen3_8_flash_next.engram":
+ *   - class Qwen3_8_FlashNextNGramEmbedding (docstring and parameters):
+ *     heads grouped by n-gram order, context reset after EOS, signed int64
+ *     wrapping hash, positive remainder per head prime, global head offsets;
+ *   - _shift_right_after_eos / _hash_input_ids: context never crosses an EOS
+ *     or a packed-segment boundary; rows of shape [batch, seq, ngram_heads];
+ *   - _lookup_ngram_ids / forward: gather of the rows, heads concatenated;
+ *   - Qwen3_8_FlashNextOwnerShardedEmbedding with process_group=None: one
+ *     local table holding every global row, no collectives; its backward is
+ *     the embedding's row-wise gradient accumulation.
+ *
+ * The page leaves the combine unprinted.  This library defines, for token t
+ * of a packed sequence and order m = 2..ngram_size,
+ *     ctx_0 = tok[t];  ctx_k = tok[t-k] if position t-k lies in t's packed
+ *     sequence and no EOS token sits in positions [t-k, t-1], else 0;
+ *     h_m = sum_{k<m} ctx_k * mults[k]            (int64, wrapping);
+ *     row[t, j] = offsets[j] + ((h_m % primes[j]) + primes[j]) % primes[j]
+ * for head j of order m = 2 + j / heads_per_ngram.  Packed sequences are
+ * given by cu_seqlens (int32 [num_seqs + 1], cu_seqlens[0] = 0,
+ * cu_seqlens[num_seqs] = num_tokens, non-decreasing); a batch of B padded
+ * rows of length S is cu_seqlens = {0, S, 2S, ...}.
+ *
+ * Conventions for every entry point:
+ *   - every tensor pointer is DEVICE memory owned by the caller; the library
+ *     never allocates on a call path (the grad scatter takes a caller
+ *     workspace); a plan owns only its host copy of the small constants;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream); calls are asynchronous on it; only ple_status synchronises;
+ *   - synchronous errors (bad arguments, alignment, workspace size, launch
+ *     failure) are returned; nothing is launched when one is returned;
+ *   - asynchronous errors found by kernels (a row id outside the table,
+ *     malformed cu_seqlens) never trap: the kernel zeroes or skips the
+ *     affected output, sets a bit in a per-device status word and carries
+ *     on; ple_status reports and clears that word.
+ *   - layouts are dense row-major; int64 rows; tables [num_rows, head_dim].
+ */
+#ifndef PLE_H_
+#define PLE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PLE_OK = 0,
+  PLE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad constants */
+  PLE_ERR_UNSUPPORTED = 2,   /* a limit of this build (see each entry) */
+  PLE_ERR_ALIGNMENT = 3,     /* pointer or row size not 16-byte aligned */
+  PLE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+  PLE_ERR_CUDA = 5,          /* CUDA runtime error; see ple_last_cuda_error */
+  PLE_ERR_BAD_ROW = 6,       /* async: a row id outside [0, num_rows) */
+  PLE_ERR_BAD_SEQLENS = 7    /* async: cu_seqlens not 0..num_tokens, or decreasing */
+} ple_status_t;
+
+typedef enum { PLE_F32 = 0, PLE_BF16 = 1 } ple_dtype_t;
+
+/* Hash and table description (constructor parameters of
+ * Qwen3_8_FlashNextNGramEmbedding and Qwen3_8_FlashNextEngramTableConfig). */
+typedef struct {
+  int32_t ngram_size;       /* largest order incl. the current token; 2..8 */
+  int32_t heads_per_ngram;  /* heads per order; H = (ngram_size-1)*heads_per_ngram <= 64 */
+  int64_t eos_id;           /* raw token id after which context resets */
+  const int64_t* mults;     /* HOST [ngram_size] signed multipliers */
+  const int64_t* primes;    /* HOST [H] per-head modulus, 2 <= p <= 2^62 */
+  const int64_t* offsets;   /* HOST [H] first global row of each head */
+  int64_t num_rows;         /* table rows; every [offset, offset+prime) inside, disjoint */
+  int32_t head_dim;         /* values per row, D */
+  ple_dtype_t table_dtype;  /* element type of the table and of lookup output */
+} ple_params_t;
+
+typedef struct ple_plan ple_plan_t;
+
+/* Validate the parameters and precompute the per-head remainder constants.
+ * Host only: touches no GPU.  Errors: PLE_ERR_INVALID_ARG (null pointers,
+ * ngram_size outside 2..8, heads_per_ngram < 1, a prime < 2 or > 2^62, a
+ * negative offset, a head range outside [0, num_rows) or overlapping
+ * another), PLE_ERR_UNSUPPORTED (H > 64), PLE_ERR_ALIGNMENT (head_dim *
+ * element size not a multiple of 16 bytes).  On success *out owns a plan
+ * that ple_plan_destroy frees. */
+ple_status_t ple_plan_create(const ple_params_t* params, ple_plan_t** out);
+void ple_plan_destroy(ple_plan_t* plan);
+int32_t ple_plan_num_heads(const ple_plan_t* plan);
+
+/* Rows of every (token, head): rows[t*H + j], int64 [num_tokens, H]
+ * (_hash_input_ids).  tokens: int64 [num_tokens]; cu_seqlens: int32
+ * [num_seqs + 1].  num_tokens == 0 is a no-op.  Errors: PLE_ERR_INVALID_ARG
+ * (null pointer, negative size, num_seqs < 1 with num_tokens > 0),
+ * PLE_ERR_ALIGNMENT (tokens or rows not 8-byte aligned), PLE_ERR_CUDA.
+ * Async: PLE_ERR_BAD_SEQLENS (rows are still written, each token using the
+ * sequence a binary search of the given array assigns it). */
+ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t num_tokens,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int64_t* rows, void* stream);
+
+/* Hash fused with the gather (forward of Qwen3_8_FlashNextNGramEmbedding):
+ * out[t, j, :] = table[row[t, j], :], out [num_tokens, H, head_dim] in the
+ * table dtype (= [tokens, H * head_dim] with heads concatenated).  The copy
+ * is exact.  rows_out, if not NULL, receives the int64 [num_tokens, H] rows
+ * (to feed ple_grad_scatter).  table and out must be 16-byte aligned.
+ * Errors as ple_hash. */
+ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t num_tokens,
+                        const int32_t* cu_seqlens, int32_t num_seqs, const void* table, void* out,
+                        int64_t* rows_out, void* stream);
+
+/* Gather precomputed rows (_lookup_ngram_ids): out[i, :] = table[rows[i], :]
+ * for i < num_hits.  A row outside [0, num_rows) yields a zero output row
+ * and the async PLE_ERR_BAD_ROW.  table and out 16-byte aligned. */
+ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits, const void* table,
+                        void* out, void* stream);
+
+/* Workspace bytes ple_grad_scatter needs for num_hits hits (0 for 0). */
+size_t ple_grad_scatter_workspace_bytes(const ple_plan_t* plan, int64_t num_hits);
+
+/* Deterministic table gradient (the embedding's backward):
+ *   table_grad[r, :] = table_grad[r, :] + S_r   for every row r hit,
+ * where S_r sums grad_out[i, :] (widened to fp32) over the hits i with
+ * rows[i] == r in this fixed order: hits in ascending i, cut into chunks of
+ * 32 consecutive hits; each chunk summed left to right from its first
+ * element; the chunk sums summed left to right from the first; one final
+ * add into table_grad.  The result is bit-identical run to run.
+ * rows int64 [num_hits]; grad_out [num_hits, head_dim] of grad_dtype;
+ * table_grad fp32 [num_rows, head_dim], accumulated into (the caller zeroes
+ * it for a fresh gradient).  Hits whose row is outside [0, num_rows) are
+ * dropped and raise the async PLE_ERR_BAD_ROW.  table_grad and grad_out
+ * 16-byte aligned; workspace 256-byte aligned.  Errors: PLE_ERR_WORKSPACE,
+ * PLE_ERR_UNSUPPORTED (num_rows >= 2^32 - 1 or num_hits >= 2^31),
+ * PLE_ERR_INVALID_ARG, PLE_ERR_ALIGNMENT, PLE_ERR_CUDA. */
+ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits,
+                              const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Same sums by fp32 atomic adds, one per hit and column: no workspace and
+ * no fixed order (results can differ in the last bits run to run).  A speed
+ * reference for the deterministic path; same argument rules. */
+ple_status_t ple_grad_scatter_atomic(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits,
+                                     const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,
+                                     void* stream);
+
+/* Synchronise `stream`, then return and clear the async status word of the
+ * current device (PLE_OK if no kernel flagged anything; otherwise the
+ * lowest-numbered flagged error).  The word is shared by all plans and
+ * streams on the device. */
+ple_status_t ple_status(void* stream);
+
+/* Text for a status code (static storage). */
+const char* ple_strerror(ple_status_t status);
+
+/* cudaError_t of the last PLE_ERR_CUDA returned on the calling thread. */
+int ple_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLE_H_ */

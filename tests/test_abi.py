@@ -1,0 +1,121 @@
+"""libple's C ABI on the host: the library loads, exports every symbol that
+include/ple.h declares, and rejects bad arguments before touching a GPU
+(every call below returns on a host check, so no device is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import hashed_gram_embedding_ple_b200 as ple
+from hashed_gram_embedding_ple_b200 import binding
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "ple.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ple_[a-z_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    lib = ple.lib()
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(binding.EXPORTS) == names
+
+
+def test_library_is_in_tree_and_built_for_sm100a():
+    path = binding.LIB_PATH
+    assert os.path.dirname(path).endswith("hashed_gram_embedding_ple_b200")
+    assert os.path.exists(path)
+
+
+def _plan(**kw):
+    args = dict(ngram_size=3, heads_per_ngram=2, eos_id=0, mults=[1, 2, 3], primes=[7, 11, 13, 17],
+                offsets=[0, 7, 18, 31], num_rows=48, head_dim=8, table_dtype=binding.torch.bfloat16)
+    args.update(kw)
+    return ple.Plan(**args)
+
+
+def test_plan_accepts_valid():
+    p = _plan()
+    assert ple.lib().ple_plan_num_heads(p.handle) == 4
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ngram_size=1, mults=[1], primes=[], offsets=[]), binding.PLE_ERR_INVALID_ARG),
+    (dict(ngram_size=9, heads_per_ngram=1, mults=[1] * 9, primes=list(range(101, 109)),
+          offsets=[0] * 8), binding.PLE_ERR_INVALID_ARG),
+    (dict(primes=[7, 1, 13, 17]), binding.PLE_ERR_INVALID_ARG),
+    (dict(offsets=[0, 6, 18, 31]), binding.PLE_ERR_INVALID_ARG),          # overlapping ranges
+    (dict(offsets=[0, 7, 18, 32]), binding.PLE_ERR_INVALID_ARG),          # past num_rows
+    (dict(offsets=[-1, 7, 18, 31]), binding.PLE_ERR_INVALID_ARG),
+    (dict(primes=[7, 11, 13, 2 ** 62 + 1], num_rows=2 ** 63 - 1), binding.PLE_ERR_INVALID_ARG),
+    (dict(head_dim=4), binding.PLE_ERR_ALIGNMENT),                          # 8-byte rows
+    (dict(head_dim=0), binding.PLE_ERR_INVALID_ARG),
+    (dict(heads_per_ngram=33, mults=[1, 2, 3], primes=[5] * 66, offsets=[0] * 66), binding.PLE_ERR_UNSUPPORTED),
+])
+def test_plan_rejects(kw, code):
+    with pytest.raises(ple.PleError) as ei:
+        _plan(**kw)
+    assert ei.value.status == code
+
+
+def test_plan_rejects_null_params():
+    lib = ple.lib()
+    out = ctypes.c_void_p()
+    assert lib.ple_plan_create(None, ctypes.byref(out)) == binding.PLE_ERR_INVALID_ARG
+    assert out.value is None
+
+
+def test_calls_reject_bad_arguments_on_host():
+    lib = ple.lib()
+    p = _plan()
+    h = p.handle
+    # empty input is a no-op
+    assert lib.ple_hash(h, None, 0, None, 0, None, None) == 0
+    assert lib.ple_lookup(h, None, 0, None, 0, None, None, None, None) == 0
+    assert lib.ple_gather(h, None, 0, None, None, None) == 0
+    assert lib.ple_grad_scatter(h, None, 0, None, 1, None, None, 0, None) == 0
+    # null / negative / misaligned
+    assert lib.ple_hash(h, None, 5, 0x1000, 1, 0x2000, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_hash(h, 0x1000, -1, 0x1000, 1, 0x2000, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_hash(h, 0x1000, 5, 0x1000, 0, 0x2000, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_hash(h, 0x1004, 5, 0x1000, 1, 0x2000, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_lookup(h, 0x1000, 5, 0x1000, 1, 0x3008, 0x4000, None, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_lookup(h, 0x1000, 5, 0x1000, 1, 0x3000, 0x4000, 0x5004, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_gather(h, 0x1000, 5, 0x3000, 0x4008, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_gather(h, None, 5, 0x3000, 0x4000, None) == binding.PLE_ERR_INVALID_ARG
+    # grad: bad dtype, workspace too small, misaligned workspace
+    assert lib.ple_grad_scatter(h, 0x1000, 5, 0x2000, 7, 0x3000, 0x4000, 1 << 20, None) == \
+        binding.PLE_ERR_INVALID_ARG
+    need = lib.ple_grad_scatter_workspace_bytes(h, 5)
+    assert need > 0
+    assert lib.ple_grad_scatter(h, 0x1000, 5, 0x2000, 1, 0x3000, 0x4000, need - 1, None) == binding.PLE_ERR_WORKSPACE
+    assert lib.ple_grad_scatter(h, 0x1000, 5, 0x2000, 1, 0x3000, None, need, None) == binding.PLE_ERR_WORKSPACE
+    assert lib.ple_grad_scatter(h, 0x1000, 5, 0x2000, 1, 0x3000, 0x4010, need, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_grad_scatter(h, 0x1000, 5, 0x2008, 1, 0x3000, 0x4000, need, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_grad_scatter(h, 0x1000, 2 ** 31, 0x2000, 1, 0x3000, 0x4000, 1 << 62, None) == \
+        binding.PLE_ERR_UNSUPPORTED
+    assert lib.ple_grad_scatter_atomic(h, None, 5, 0x2000, 1, 0x3000, None) == binding.PLE_ERR_INVALID_ARG
+
+
+def test_workspace_grows_with_hits():
+    p = _plan(head_dim=128)
+    a = ple.workspace_bytes(p, 1000)
+    b = ple.workspace_bytes(p, 100000)
+    assert 0 < a < b
+    assert ple.workspace_bytes(p, 0) == 0
+    # keys/values double buffers plus chunk-sum slots dominate: roughly 16 B + 2*D*4/32 B per hit
+    assert b >= 100000 * (16 + 2 * 128 * 4 // 32)
+
+
+def test_strerror_covers_codes():
+    lib = ple.lib()
+    for c in range(8):
+        assert lib.ple_strerror(c)
+    assert b"unknown" in lib.ple_strerror(99)

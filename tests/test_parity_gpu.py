@@ -1,0 +1,219 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Rows, gathered values and the deterministic gradient must be bit-identical
+to the oracle; the atomic gradient variant is held to a relative 1e-5.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import hashed_gram_embedding_ple_b200 as ple
+from gpu_util import (custom_workload, dev_i32, dev_i64, host_grad, small_table, torch_to_values,
+                      values_to_torch)
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_rows(w):
+    return oracle.rows(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
+                       w.offsets)
+
+
+def run_forward(w, dev):
+    plan = ple.Plan.from_workload(w)
+    tok, cu = dev_i64(w.tokens, dev), dev_i32(w.cu_seqlens, dev)
+    host_table, table = small_table(w, dev)
+    rows = ple.ple_hash(plan, tok, cu)
+    out, rows_out = ple.ple_lookup(plan, tok, cu, table, save_rows=True)
+    gathered = ple.ple_gather(plan, rows, table)
+    assert ple.ple_status() == ple.PLE_OK
+    return plan, host_table, rows.cpu().numpy(), rows_out.cpu().numpy(), torch_to_values(out), \
+        torch_to_values(gathered)
+
+
+def check_forward(w, dev):
+    plan, host_table, rows, rows_out, out, gathered = run_forward(w, dev)
+    ref_rows = oracle_rows(w)
+    np.testing.assert_array_equal(rows, ref_rows)
+    np.testing.assert_array_equal(rows_out, ref_rows)
+    ref_out = oracle.gather(ref_rows, host_table)
+    assert out.shape == ref_out.shape
+    np.testing.assert_array_equal(out, ref_out)
+    np.testing.assert_array_equal(gathered, ref_out)
+    return ref_rows
+
+
+def check_backward(w, dev, rows_np, prefill=None):
+    plan = ple.Plan.from_workload(w)
+    N = rows_np.size
+    g_host = host_grad(w, N)
+    g = values_to_torch(g_host, w.grad_dtype).to(dev)
+    rows = dev_i64(rows_np.reshape(-1), dev)
+    base = np.zeros((w.num_rows, w.head_dim), np.float32) if prefill is None else prefill.copy()
+    tg = torch.from_numpy(base.copy()).to(dev)
+    ple.ple_grad_scatter(plan, rows, g, tg)
+    assert ple.ple_status() == ple.PLE_OK
+    ref = oracle.grad_apply(rows_np.reshape(-1), g_host, base.copy())
+    got = tg.cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # run to run: bit-identical again
+    tg2 = torch.from_numpy(base.copy()).to(dev)
+    ple.ple_grad_scatter(plan, rows, g, tg2)
+    assert torch.equal(tg2.view(torch.int32), tg.view(torch.int32))
+    # atomic variant: the same sums in an unspecified order.  Relative error
+    # 1e-5 is measured against the magnitude sum |base| + sum |g| of each
+    # element (the scale of any fp32 reordering error), since the sum itself
+    # may cancel to near zero.
+    tg3 = torch.from_numpy(base.copy()).to(dev)
+    ple.ple_grad_scatter_atomic(plan, rows, g, tg3)
+    torch.cuda.synchronize()
+    g32 = torch.from_numpy(g_host.astype(np.float32) if w.grad_dtype == synth.DTYPE_F32 else
+                           synth.bf16_bits_to_f32(g_host)).double()
+    mag = torch.from_numpy(np.abs(base)).double().index_add_(0, torch.from_numpy(rows_np.reshape(-1)), g32.abs())
+    err = np.abs(tg3.cpu().numpy().astype(np.float64) - ref.astype(np.float64))
+    assert np.all(err <= 1e-5 * mag.numpy() + 1e-30)
+
+
+# ---------------------------------------------------------------------------
+
+def test_tiny_forward_backward(cuda_device):
+    w = synth.tiny(0)
+    rows = check_forward(w, cuda_device)
+    check_backward(w, cuda_device, rows)
+
+
+@pytest.mark.parametrize("n,G,D,dt", [
+    (2, 1, 8, synth.DTYPE_BF16),     # 16-byte rows
+    (3, 3, 48, synth.DTYPE_F32),     # 192-byte rows: 12 vectors, not a power of two
+    (4, 2, 24, synth.DTYPE_BF16),    # 48-byte rows: 3 vectors
+    (4, 5, 128, synth.DTYPE_BF16),
+    (5, 4, 64, synth.DTYPE_F32),
+    (8, 1, 256, synth.DTYPE_BF16),   # largest order
+    (3, 32, 32, synth.DTYPE_F32),    # 64 heads
+])
+def test_ragged_multi_tile(cuda_device, n, G, D, dt):
+    rng = np.random.default_rng(100 + n * 10 + G)
+    lens = [1, 0, 37, 5000 - 38 - 13, 13]  # several tiles, a ragged tail, an empty and a 1-token sequence
+    T = sum(lens)
+    tok = rng.integers(0, 50, T)  # small vocabulary: many repeats and many EOS (id 0)
+    mults = synth.signed_mults(n, rng)
+    primes = synth.consecutive_primes(int(rng.integers(50, 400)), (n - 1) * G)
+    w = custom_workload("ragged", tok, synth.cu_seqlens_from_lengths(lens), n, G, 0, mults, primes, D, dt, dt,
+                        seed=n)
+    rows = check_forward(w, cuda_device)
+    check_backward(w, cuda_device, rows)
+
+
+def test_production_constants_forward(cuda_device):
+    from conftest import read_golden_blocks
+
+    _, g = read_golden_blocks("production_constants.txt")
+    primes = synth.consecutive_primes(20_000_000, 16)
+    rng = np.random.default_rng(1)
+    T = 3000
+    tok = rng.integers(0, 248_320, T)
+    tok[rng.random(T) < 0.02] = g["eos_token_id"][0]
+    w = custom_workload("prod", tok, [0, 1234, T], 3, 8, g["eos_token_id"][0], g["multipliers"], primes, 8,
+                        synth.DTYPE_BF16)
+    plan = ple.Plan.from_workload(w)
+    rows = ple.ple_hash(plan, dev_i64(w.tokens, cuda_device), dev_i32(w.cu_seqlens, cuda_device))
+    np.testing.assert_array_equal(rows.cpu().numpy(), oracle_rows(w))
+
+
+def test_edge_cases(cuda_device):
+    dev = cuda_device
+    rng = np.random.default_rng(3)
+    mults = [2 ** 63 - 1, -(2 ** 63), 12345]
+    # all EOS; single token; alternating EOS; many 1-token sequences
+    cases = [
+        (np.zeros(70, np.int64), [0, 70]),
+        (np.array([5], np.int64), [0, 1]),
+        (np.tile([0, 7], 40), [0, 80]),
+        (rng.integers(0, 5, 100), list(range(0, 101))),
+        (rng.integers(0, 5, 64), [0, 0, 0, 32, 32, 64, 64]),
+    ]
+    for k, (tok, cu) in enumerate(cases):
+        w = custom_workload(f"edge{k}", tok, cu, 3, 2, 0, mults, [5, 7, 11, 13], 8, synth.DTYPE_F32)
+        rows = check_forward(w, dev)
+        check_backward(w, dev, rows)
+
+
+def test_empty_inputs(cuda_device):
+    w = synth.tiny(0)
+    plan = ple.Plan.from_workload(w)
+    tok = torch.empty(0, dtype=torch.int64, device=cuda_device)
+    cu = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    _, table = small_table(w, cuda_device)
+    assert ple.ple_hash(plan, tok, cu).shape == (0, 4)
+    assert ple.ple_lookup(plan, tok, cu, table).shape == (0, 4, 32)
+    tg = torch.zeros(w.num_rows, w.head_dim, device=cuda_device)
+    ple.ple_grad_scatter(plan, tok, torch.empty(0, 32, device=cuda_device), tg)
+    assert ple.ple_status() == ple.PLE_OK and not tg.any()
+
+
+def test_gradient_chunk_boundaries(cuda_device):
+    """Rows hit exactly 1, 31, 32, 33, 64, 65, 1000 and 5000 times, interleaved."""
+    rng = np.random.default_rng(5)
+    counts = {3: 1, 10: 31, 11: 32, 12: 33, 20: 64, 21: 65, 30: 1000, 31: 5000}
+    rows = np.concatenate([np.full(c, r) for r, c in counts.items()] + [rng.integers(0, 40, 3000)])
+    rows = rng.permutation(rows)
+    w = custom_workload("chunks", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [41], 64, synth.DTYPE_F32,
+                        synth.DTYPE_BF16)
+    prefill = synth.dense_values(9, 41 * 64, 0.5, synth.DTYPE_F32).reshape(41, 64)
+    check_backward(w, cuda_device, rows, prefill=prefill)
+
+
+@pytest.mark.parametrize("D,gdt", [(32, synth.DTYPE_F32), (64, synth.DTYPE_BF16), (128, synth.DTYPE_BF16),
+                                   (256, synth.DTYPE_F32), (40, synth.DTYPE_BF16), (200, synth.DTYPE_F32)])
+def test_gradient_many_tiles(cuda_device, D, gdt):
+    """Zipf-heavy rows over several sort tiles and a ragged tail."""
+    rng = np.random.default_rng(D)
+    R = 70_001
+    N = 3 * 4096 + 1234
+    rows = synth.zipf_ids(N, 1.3, R, rng)
+    w = custom_workload("gtiles", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [R], D, synth.DTYPE_F32, gdt)
+    check_backward(w, cuda_device, rows)
+
+
+def test_bad_rows_flagged(cuda_device):
+    dev = cuda_device
+    w = synth.tiny(0)
+    plan = ple.Plan.from_workload(w)
+    host_table, table = small_table(w, dev)
+    rows_np = np.array([5, -1, 24591, 24592, 2 ** 40, 7], np.int64)
+    out = ple.ple_gather(plan, dev_i64(rows_np, dev), table)
+    assert ple.ple_status() == ple.PLE_ERR_BAD_ROW
+    assert ple.ple_status() == ple.PLE_OK  # cleared
+    o = out.cpu().numpy()
+    np.testing.assert_array_equal(o[[0, 2, 5]], host_table[[5, 24591, 7]])
+    assert not o[[1, 3, 4]].any()
+    # gradient: bad hits dropped, the rest exact
+    g_host = host_grad(w, len(rows_np))
+    tg = torch.zeros(w.num_rows, w.head_dim, device=dev)
+    ple.ple_grad_scatter(plan, dev_i64(rows_np, dev), values_to_torch(g_host, w.grad_dtype).to(dev), tg)
+    assert ple.ple_status() == ple.PLE_ERR_BAD_ROW
+    good = np.array([0, 2, 5])
+    ref = oracle.grad_apply(rows_np[good], g_host[good], np.zeros((w.num_rows, w.head_dim), np.float32))
+    np.testing.assert_array_equal(tg.cpu().numpy(), ref)
+
+
+def test_malformed_seqlens_flagged(cuda_device):
+    dev = cuda_device
+    w = synth.tiny(0)
+    plan = ple.Plan.from_workload(w)
+    tok = dev_i64(w.tokens, dev)
+    for bad in ([0, 200, 100, 256], [1, 100, 256], [0, 100, 250]):
+        rows = ple.ple_hash(plan, tok, dev_i32(bad, dev))
+        assert ple.ple_status() == ple.PLE_ERR_BAD_SEQLENS
+        r = rows.cpu().numpy()
+        assert np.all(r >= w.offsets) and np.all(r < w.offsets + w.primes)
+
+
+def test_library_loaded_from_tree(cuda_device):
+    import os
+
+    ple.lib()
+    maps = open("/proc/self/maps").read()
+    assert os.path.realpath(ple.binding.LIB_PATH) in maps
