@@ -31,15 +31,13 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
+constexpr int kSortItems = 4;
 constexpr int kSortTile = kSortThreads * kSortItems;  // keys per sort tile
 constexpr int kRadix = 256;
 constexpr int kWarpsPerSortBlock = kSortThreads / 32;
 constexpr int kChunk = 32;
 constexpr uint32_t kNoKey = 0xffffffffu;  // past the end; never a real key
-constexpr int kScanThreads = 1024;
 constexpr int kFoldThreads = 256;
-constexpr int kFoldBatch = 8;             // grad rows loaded ahead in the fold
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -49,7 +47,17 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 // ---------------------------------------------------------------------------
 // radix sort
+//
+// Tiles of 4096 keys; inside a tile warp w owns positions [512w, 512w+512),
+// read in 16 rounds of 32, so (warp, round, lane) is the tile order.
+// Histograms are stored tile-major, hist[tile][digit].  Tiles form groups of
+// 32: the last block of a group to finish its histogram (atomic ticket, no
+// waiting) turns the group's histograms into in-group exclusive prefixes and
+// writes the group's digit totals.  A scatter block then derives its global
+// digit offsets from the (few) group totals itself, so no device-wide scan
+// kernel is needed.
 // ---------------------------------------------------------------------------
+constexpr int kTilesPerGroup = 32;
 
 // Warp-aggregated shared-memory histogram update for one key per lane.
 __device__ __forceinline__ void hist_add(uint32_t* h, bool valid, uint32_t digit) {
@@ -57,18 +65,103 @@ __device__ __forceinline__ void hist_add(uint32_t* h, bool valid, uint32_t digit
   if (valid && (peers & lanemask_lt()) == 0) atomicAdd(&h[digit], __popc(peers));
 }
 
+__device__ __forceinline__ int64_t tile_pos(int64_t tile, int warp, int r, int lane) {
+  return tile * kSortTile + warp * (kSortTile / kWarpsPerSortBlock) + r * 32 + lane;
+}
+
+// Block-wide exclusive sum over the 256 threads (one value per thread).
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t x, uint32_t* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = x;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, incl, d);
+    if (lane >= d) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int w = 0; w < warp; ++w) before += warp_tot[w];
+  return before + incl - x;
+}
+
+// Publish this block's histogram.  The last block of a group of 32 tiles to
+// arrive (atomic ticket, nobody waits) turns the group's histograms into
+// in-group exclusive prefixes and writes the group's digit totals; the last
+// group to finish then turns the group totals into gbase[group][digit] =
+// (keys of smaller digits) + (keys of this digit in earlier groups).  A
+// scatter block's global offset for digit d is gbase[its group][d] +
+// hist[its tile][d].
+__device__ void publish_histogram(const uint32_t* h, uint32_t* __restrict__ hist, uint32_t* __restrict__ gtot,
+                                  unsigned int* __restrict__ tickets, int num_tiles) {
+  __shared__ bool is_last;
+  __shared__ uint32_t warp_tot[kWarpsPerSortBlock];
+  const int tile = blockIdx.x, d = threadIdx.x;
+  const int ngroups = (num_tiles + kTilesPerGroup - 1) / kTilesPerGroup;
+  unsigned int* group_done = tickets + ngroups;  // one more counter after the per-group tickets
+  hist[static_cast<int64_t>(tile) * kRadix + d] = h[d];
+  __threadfence();
+  __syncthreads();
+  const int g = tile / kTilesPerGroup;
+  const int first = g * kTilesPerGroup;
+  const int n = min(kTilesPerGroup, num_tiles - first);
+  if (threadIdx.x == 0) is_last = atomicAdd(&tickets[g], 1u) == static_cast<unsigned>(n - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  {
+    uint32_t v[kTilesPerGroup];
+    uint32_t* col = hist + static_cast<int64_t>(first) * kRadix + d;
+#pragma unroll
+    for (int k = 0; k < kTilesPerGroup; ++k) v[k] = k < n ? __ldcg(col + k * kRadix) : 0;  // all loads first
+    uint32_t run = 0;
+#pragma unroll
+    for (int k = 0; k < kTilesPerGroup; ++k) {
+      if (k < n) col[k * kRadix] = run;
+      run += v[k];
+    }
+    gtot[static_cast<int64_t>(g) * kRadix + d] = run;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tickets[g] = 0;  // ready for the next pass / call
+    is_last = atomicAdd(group_done, 1u) == static_cast<unsigned>(ngroups - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // exclusive prefix over groups per digit, then the digit base over digits
+  uint32_t total = 0;
+#pragma unroll 8
+  for (int k = 0; k < ngroups; ++k) total += __ldcg(gtot + static_cast<int64_t>(k) * kRadix + d);
+  const uint32_t digit_base = block_exclusive_sum(total, warp_tot);
+  uint32_t run = digit_base;
+  for (int k0 = 0; k0 < ngroups; k0 += 8) {
+    uint32_t v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = k0 + k < ngroups ? __ldcg(gtot + static_cast<int64_t>(k0 + k) * kRadix + d) : 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k0 + k < ngroups) gtot[static_cast<int64_t>(k0 + k) * kRadix + d] = run;
+      run += v[k];
+    }
+  }
+  if (threadIdx.x == 0) *group_done = 0;
+}
+
 __global__ void __launch_bounds__(kSortThreads)
 keys_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, uint32_t* __restrict__ keys,
-            uint32_t* __restrict__ hist, int num_tiles, int* __restrict__ mc_count, unsigned int* status) {
+            uint32_t* __restrict__ hist, uint32_t* __restrict__ gtot, unsigned int* __restrict__ tickets,
+            int num_tiles, unsigned int* status) {
   __shared__ uint32_t h[kRadix];
   h[threadIdx.x] = 0;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *mc_count = 0;
   __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bool bad = false;
 #pragma unroll 4
   for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * kSortThreads + threadIdx.x;
+    const int64_t i = tile_pos(blockIdx.x, warp, r, lane);
     const bool valid = i < N;
     uint32_t key = 0;
     if (valid) {
@@ -82,125 +175,83 @@ keys_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, uint3
   }
   if (bad) raise_flag(status, PLE_ERR_BAD_ROW);
   __syncthreads();
-  hist[threadIdx.x * num_tiles + blockIdx.x] = h[threadIdx.x];
+  publish_histogram(h, hist, gtot, tickets, num_tiles);
 }
 
 __global__ void __launch_bounds__(kSortThreads)
 hist_kernel(const uint32_t* __restrict__ keys, int64_t N, int shift, uint32_t* __restrict__ hist,
-            int num_tiles) {
+            uint32_t* __restrict__ gtot, unsigned int* __restrict__ tickets, int num_tiles) {
   __shared__ uint32_t h[kRadix];
   h[threadIdx.x] = 0;
   __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
-#pragma unroll 4
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t key[kSortItems];
+#pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * kSortThreads + threadIdx.x;
-    const bool valid = i < N;
-    const uint32_t key = valid ? keys[i] : 0;
-    hist_add(h, valid, (key >> shift) & (kRadix - 1));
+    const int64_t i = tile_pos(blockIdx.x, warp, r, lane);
+    key[r] = i < N ? keys[i] : 0;
   }
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r)
+    hist_add(h, tile_pos(blockIdx.x, warp, r, lane) < N, (key[r] >> shift) & (kRadix - 1));
   __syncthreads();
-  hist[threadIdx.x * num_tiles + blockIdx.x] = h[threadIdx.x];
+  publish_histogram(h, hist, gtot, tickets, num_tiles);
 }
 
-// Exclusive scan, in place, of M counters laid out digit-major
-// ([digit][tile]), by one block: each thread owns a contiguous run.
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(uint32_t* __restrict__ a, int M) {
-  __shared__ uint32_t warp_tot[kScanThreads / 32];
-  const int per = (M + kScanThreads - 1) / kScanThreads;
-  const int beg = min(M, threadIdx.x * per), end = min(M, beg + per);
-  uint32_t s = 0;
-  for (int i = beg; i < end; ++i) s += a[i];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t incl = s;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t y = __shfl_up_sync(kFull, incl, d);
-    if (lane >= d) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = warp_tot[lane];
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t y = __shfl_up_sync(kFull, w, d);
-      if (lane >= d) w += y;
-    }
-    warp_tot[lane] = w;  // inclusive
-  }
-  __syncthreads();
-  uint32_t run = incl - s + (warp > 0 ? warp_tot[warp - 1] : 0);
-  for (int i = beg; i < end; ++i) {
-    const uint32_t v = a[i];
-    a[i] = run;
-    run += v;
-  }
-}
-
-// Stable rank-and-scatter of one 4096-key tile.  Keys are held striped
-// (item r of thread x is tile position r*256 + x), so the order
-// (r, warp, lane) is the tile order.  Per (item round, warp, digit) counts
-// go to shared memory; one pass per digit turns them into exclusive
-// offsets; the destination is the tile's scanned global digit offset plus
-// that offset plus the rank among equal digits inside the warp.
-constexpr size_t kScatterSmem =
-    sizeof(uint16_t) * kSortItems * kWarpsPerSortBlock * kRadix + sizeof(uint32_t) * kRadix;
-
+// Stable rank-and-scatter of one tile.  Rank of a key = its tile's global
+// digit offset + the keys of that digit in earlier warps of the tile + the
+// keys of that digit earlier in its own warp (running per-warp counts,
+// updated round by round after every lane has read them).
 template <bool kIdentityVals>
 __global__ void __launch_bounds__(kSortThreads)
 scatter_kernel(const uint32_t* __restrict__ kin, const uint32_t* __restrict__ vin, uint32_t* __restrict__ kout,
-               uint32_t* __restrict__ vout, const uint32_t* __restrict__ offs, int64_t N, int shift,
-               int num_tiles) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint16_t* cnt = reinterpret_cast<uint16_t*>(smem);  // [items][warps][radix]
-  uint32_t* tile_base = reinterpret_cast<uint32_t*>(cnt + kSortItems * kWarpsPerSortBlock * kRadix);
-  const int warp = threadIdx.x >> 5;
-  {
-    uint32_t* c32 = reinterpret_cast<uint32_t*>(cnt);
-    constexpr int words = kSortItems * kWarpsPerSortBlock * kRadix / 2;
-#pragma unroll 4
-    for (int k = threadIdx.x; k < words; k += kSortThreads) c32[k] = 0;
-  }
-  tile_base[threadIdx.x] = offs[threadIdx.x * num_tiles + blockIdx.x];
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
+               uint32_t* __restrict__ vout, const uint32_t* __restrict__ hist, const uint32_t* __restrict__ gtot,
+               int64_t N, int shift, int num_tiles) {
+  __shared__ uint32_t wh[kWarpsPerSortBlock][kRadix];
+  __shared__ uint32_t tile_base[kRadix];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, d = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int g = tile / kTilesPerGroup;
+
   uint32_t key[kSortItems], val[kSortItems];
-  uint8_t rank[kSortItems];
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * kSortThreads + threadIdx.x;
+    const int64_t i = tile_pos(tile, warp, r, lane);
     key[r] = i < N ? kin[i] : kNoKey;
     val[r] = i < N ? (kIdentityVals ? static_cast<uint32_t>(i) : vin[i]) : 0;
   }
+  tile_base[d] = gtot[static_cast<int64_t>(g) * kRadix + d] + hist[static_cast<int64_t>(tile) * kRadix + d];
+#pragma unroll
+  for (int w = 0; w < kWarpsPerSortBlock; ++w) wh[w][d] = 0;
   __syncthreads();
+  uint16_t rank[kSortItems];
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * kSortThreads + threadIdx.x;
-    const bool valid = i < N;
+    const bool valid = tile_pos(tile, warp, r, lane) < N;
     const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
     const unsigned peers = __match_any_sync(kFull, valid ? digit : 0x100u);
     const unsigned lower = __popc(peers & lanemask_lt());
-    rank[r] = static_cast<uint8_t>(lower);
-    if (valid && lower == 0) cnt[(r * kWarpsPerSortBlock + warp) * kRadix + digit] = __popc(peers);
+    rank[r] = valid ? static_cast<uint16_t>(wh[warp][digit] + lower) : 0;
+    __syncwarp();
+    if (valid && lower == 0) wh[warp][digit] += __popc(peers);
+    __syncwarp();
   }
   __syncthreads();
   {
-    const int d = threadIdx.x;
     uint32_t run = 0;
-    for (int rw = 0; rw < kSortItems * kWarpsPerSortBlock; ++rw) {
-      const uint32_t c = cnt[rw * kRadix + d];
-      cnt[rw * kRadix + d] = static_cast<uint16_t>(run);
+#pragma unroll
+    for (int w = 0; w < kWarpsPerSortBlock; ++w) {
+      const uint32_t c = wh[w][d];
+      wh[w][d] = run;
       run += c;
     }
   }
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = base + r * kSortThreads + threadIdx.x;
-    if (i < N) {
+    if (tile_pos(tile, warp, r, lane) < N) {
       const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-      const uint32_t dst =
-          tile_base[digit] + cnt[(r * kWarpsPerSortBlock + warp) * kRadix + digit] + rank[r];
+      const uint32_t dst = tile_base[digit] + wh[warp][digit] + rank[r];
       if (dst < N) {  // always true when the counts are consistent
         kout[dst] = key[r];
         vout[dst] = val[r];
@@ -339,97 +390,268 @@ __device__ int64_t find_run_start(const uint32_t* __restrict__ K, int64_t p, uin
   return hi;
 }
 
-// Level 1: one warp per window of 32 sorted positions.
-template <int CPL, bool BF16>
-__global__ void __launch_bounds__(kFoldThreads)
-fold_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
-            const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
-            int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5;
-  const int64_t p0 = w * 32;
-  if (p0 >= N) return;
-  const int64_t pa = p0 + lane, pb = p0 + 32 + lane;
-  const uint32_t kA = pa < N ? K[pa] : kNoKey;
-  const uint32_t kB = pb < N ? K[pb] : kNoKey;
-  const uint32_t iA = pa < N ? I[pa] : 0;
-  const uint32_t iB = pb < N ? I[pb] : 0;
-  const uint32_t k_before = p0 > 0 ? K[p0 - 1] : kNoKey;
-  uint32_t prevA = __shfl_up_sync(kFull, kA, 1);
-  uint32_t prevB = __shfl_up_sync(kFull, kB, 1);
-  const uint32_t kA31 = __shfl_sync(kFull, kA, 31);
-  if (lane == 0) {
-    prevA = k_before;
-    prevB = kA31;
-  }
-  const bool headA = pa < N && kA != prevA;
-  const bool headB = pb < N && kB != prevB;
-  const uint64_t hm = static_cast<uint64_t>(__ballot_sync(kFull, headA)) |
-                      (static_cast<uint64_t>(__ballot_sync(kFull, headB)) << 32);
-  const uint32_t key0 = __shfl_sync(kFull, kA, 0);
-  const int64_t s0 = (hm & 1ull) ? p0 : find_run_start(K, p0, key0);
-
-  auto run_start = [&](int idx) -> int64_t {  // first position of the run holding p0 + idx
+// Level 1 works on windows of 32 sorted positions, one warp per window.
+// One round trip brings the window's keys and hit indices, the next 32 keys
+// (a chunk that starts in this window may end in the next) and the previous
+// 32 keys (to find where the run holding the window's first position starts;
+// only runs longer than 32 need the search).  The warp folds the chunks that
+// START in its window: positions [a, b) relative to p0, b being the first
+// chunk start of the next window (or the end).
+struct Window {
+  uint64_t hm;   // run starts among positions p0 .. p0+63
+  uint64_t cm;   // chunk starts among positions p0 .. p0+63
+  int64_t p0, s0;
+  int a, b;
+  uint32_t kA, kB, iA, iB;
+  __device__ int64_t run_start(int idx) const {  // first position of the run holding p0 + idx
     const uint64_t le = hm & (idx >= 63 ? ~0ull : ((2ull << idx) - 1));
     return le ? p0 + (63 - __clzll(le)) : s0;
-  };
-  const bool csA = pa < N && ((pa - run_start(lane)) & (kChunk - 1)) == 0;
-  const bool csB = pb < N && ((pb - run_start(32 + lane)) & (kChunk - 1)) == 0;
-  const uint64_t cm = static_cast<uint64_t>(__ballot_sync(kFull, csA)) |
-                      (static_cast<uint64_t>(__ballot_sync(kFull, csB)) << 32);
+  }
+  __device__ uint32_t key_at(int e) const {  // warp-uniform e in [0, 64)
+    const uint32_t ka = __shfl_sync(kFull, kA, e & 31), kb = __shfl_sync(kFull, kB, e & 31);
+    return e < 32 ? ka : kb;
+  }
+};
+
+__device__ __forceinline__ bool window_setup(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
+                                             int64_t N, int64_t w, Window& W) {
+  const int lane = threadIdx.x & 31;
+  const int64_t p0 = w * 32;
+  const int64_t pa = p0 + lane, pb = p0 + 32 + lane, pc = p0 - 32 + lane;
+  W.p0 = p0;
+  W.kA = pa < N ? K[pa] : kNoKey;
+  W.kB = pb < N ? K[pb] : kNoKey;
+  const uint32_t kC = p0 > 0 ? K[pc] : kNoKey;  // p0 is a multiple of 32, so pc >= 0 here
+  W.iA = pa < N ? I[pa] : 0;
+  W.iB = pb < N ? I[pb] : 0;
+  uint32_t prevA = __shfl_up_sync(kFull, W.kA, 1);
+  uint32_t prevB = __shfl_up_sync(kFull, W.kB, 1);
+  const uint32_t kA31 = __shfl_sync(kFull, W.kA, 31);
+  const uint32_t kC31 = __shfl_sync(kFull, kC, 31);
+  if (lane == 0) {
+    prevA = kC31;
+    prevB = kA31;
+  }
+  const bool headA = pa < N && W.kA != prevA;
+  const bool headB = pb < N && W.kB != prevB;
+  W.hm = static_cast<uint64_t>(__ballot_sync(kFull, headA)) |
+         (static_cast<uint64_t>(__ballot_sync(kFull, headB)) << 32);
+  const uint32_t key0 = __shfl_sync(kFull, W.kA, 0);
+  W.s0 = p0;
+  if (!(W.hm & 1ull)) {
+    // p0 > 0 here; the run started among the previous 32 positions unless
+    // all of them hold key0
+    const unsigned differ = __ballot_sync(kFull, kC != key0);
+    W.s0 = differ ? p0 - 32 + (32 - __clz(differ)) : find_run_start(K, p0 - 32, key0);
+  }
+  const bool csA = pa < N && ((pa - W.run_start(lane)) & (kChunk - 1)) == 0;
+  const bool csB = pb < N && ((pb - W.run_start(32 + lane)) & (kChunk - 1)) == 0;
+  W.cm = static_cast<uint64_t>(__ballot_sync(kFull, csA)) | (static_cast<uint64_t>(__ballot_sync(kFull, csB)) << 32);
   // A window may hold no chunk start only at the tail, when its positions
   // finish a chunk that started in the previous window (folded there).
-  if ((cm & 0xffffffffull) == 0) return;
-  const int a = __ffsll(static_cast<long long>(cm & 0xffffffffull)) - 1;
-  const uint32_t hiw = static_cast<uint32_t>(cm >> 32);
-  const int b = hiw ? 32 + __ffs(hiw) - 1 : static_cast<int>(N - p0);
+  if ((W.cm & 0xffffffffull) == 0) return false;
+  W.a = __ffsll(static_cast<long long>(W.cm & 0xffffffffull)) - 1;
+  const uint32_t hiw = static_cast<uint32_t>(W.cm >> 32);
+  W.b = hiw ? 32 + __ffs(hiw) - 1 : static_cast<int>(N - p0);
+  return true;
+}
 
-  Cols<CPL> acc;
+// Bookkeeping of a finished chunk [c, nxt) (relative positions) whose sum the
+// calling lanes hold: returns true if the chunk is a whole run (the caller
+// adds it into table_grad), false if its sum goes to a chunk-sum slot
+// (returned in *slot); lane `leader` records heavy-run metadata.
+__device__ __forceinline__ bool chunk_is_whole_run(const Window& W, int c, int nxt, int64_t N, bool leader,
+                                                   int64_t* slot, int* __restrict__ mc_len,
+                                                   int* __restrict__ mc_list, int* __restrict__ mc_count) {
+  const bool is_head = (W.hm >> c) & 1ull;
+  const bool run_ends = (W.p0 + nxt >= N) || ((W.hm >> nxt) & 1ull);
+  if (is_head && run_ends) return true;
+  const int64_t pos = W.p0 + c;
+  *slot = 2 * (pos >> 5) + (is_head ? 1 : 0);
+  if (leader) {
+    if (is_head) mc_list[atomicAdd(mc_count, 1)] = static_cast<int>(pos);
+    if (run_ends) {
+      const int64_t s = W.run_start(c);
+      mc_len[s >> 5] = static_cast<int>(W.p0 + nxt - s);
+    }
+  }
+  return false;
+}
+
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <bool BF16>
+__device__ __forceinline__ void unpack16(const uint4& y, float* v) {
+  if constexpr (BF16) {
+    v[0] = bf16_lo(y.x); v[1] = bf16_hi(y.x); v[2] = bf16_lo(y.y); v[3] = bf16_hi(y.y);
+    v[4] = bf16_lo(y.z); v[5] = bf16_hi(y.z); v[6] = bf16_lo(y.w); v[7] = bf16_hi(y.w);
+  } else {
+    v[0] = __uint_as_float(y.x); v[1] = __uint_as_float(y.y);
+    v[2] = __uint_as_float(y.z); v[3] = __uint_as_float(y.w);
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+constexpr int kWideWarps = 4;  // warps per block of the wide fold
+constexpr int kWideLoads = 8;  // 16-byte async copies per lane per batch
+
+// Wide fold: a grad row spans L lanes that each copy 16 bytes, so one
+// instruction fetches 32/L rows.  A batch of rows is staged in shared memory
+// by asynchronous copies (no registers held while they are in flight).  A run
+// of a single hit is added into table_grad by the lane group that fetched it.
+// Hits of longer runs are folded in order: every L-lane group keeps the same
+// running chunk sum (lane `sub` of a group owns CPLN = 16/elem columns) and
+// adds row after row from the staging buffer; the groups write finished
+// chunks in turn.
+template <int L, bool BF16>
+__global__ void __launch_bounds__(kWideWarps * 32, 8)
+fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
+                 const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
+                 int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
+  constexpr int RPI = 32 / L;                                            // rows per copy instruction
+  constexpr int CPLN = BF16 ? 8 : 4;                                     // fp32 columns per lane
+  constexpr int BATCH = kWideLoads * RPI < 64 ? kWideLoads * RPI : 64;   // hits per batch
+  constexpr int LOADS = BATCH / RPI;                                     // copies per lane per batch
+  __shared__ uint4 stage[kWideWarps][kWideLoads][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / L, sub = lane % L;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWideWarps + warp;
+  if (w * 32 >= N) return;
+  Window W;
+  if (!window_setup(K, I, N, w, W)) return;
+  const size_t row_bytes = static_cast<size_t>(D) * (BF16 ? 2 : 4);
+  const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
+  // positions holding a run of exactly one hit
+  const uint64_t next_is_head = (W.hm >> 1) | (W.p0 + 63 >= N ? (1ull << (N - 1 - W.p0)) : 0ull);
+  const uint64_t single = W.hm & next_is_head;
+
+  float acc[CPLN];
 #pragma unroll
-  for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = 0.f;
-  int c = a;  // current chunk start (relative)
-  for (int e0 = a; e0 < b; e0 += kFoldBatch) {
-    Cols<CPL> g[kFoldBatch];
+  for (int k = 0; k < CPLN; ++k) acc[k] = 0.f;
+  int c = W.a, turn = 0;
+  for (int e0 = W.a; e0 < W.b; e0 += BATCH) {
 #pragma unroll
-    for (int u = 0; u < kFoldBatch; ++u) {
+    for (int s = 0; s < LOADS; ++s) {
+      const int e = e0 + s * RPI + grp;
+      const int src = e & 31;
+      const uint32_t ia = __shfl_sync(kFull, W.iA, src), ib = __shfl_sync(kFull, W.iB, src);
+      if (e < W.b) cp_async16(&stage[warp][s][lane], gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
+    }
+    cp_async_wait_all();
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < LOADS; ++s) {
+      const int e = e0 + s * RPI + grp;
+      const int src = e & 31;
+      const uint32_t ka = __shfl_sync(kFull, W.kA, src), kb = __shfl_sync(kFull, W.kB, src);
+      const uint32_t key = e < 32 ? ka : kb;
+      if (e < W.b && ((single >> e) & 1ull) && key != bad_key) {
+        float v[CPLN];
+        unpack16<BF16>(stage[warp][s][lane], v);
+        float* dst = table_grad + static_cast<int64_t>(key) * D + sub * CPLN;
+#pragma unroll
+        for (int k = 0; k < CPLN; k += 4) red_add4(dst + k, v[k], v[k + 1], v[k + 2], v[k + 3]);
+      }
+    }
+    const int nb = min(BATCH, W.b - e0);
+    uint64_t multi = (~single >> e0) & (nb >= 64 ? ~0ull : ((1ull << nb) - 1));
+    while (multi) {
+      const int t = __ffsll(static_cast<long long>(multi)) - 1;
+      multi &= multi - 1;
+      const int e = e0 + t;
+      float v[CPLN];
+      unpack16<BF16>(stage[warp][t / RPI][sub + L * (t % RPI)], v);
+      if ((W.cm >> e) & 1ull) {
+        c = e;
+#pragma unroll
+        for (int k = 0; k < CPLN; ++k) acc[k] = v[k];
+      } else {
+#pragma unroll
+        for (int k = 0; k < CPLN; ++k) acc[k] = acc[k] + v[k];
+      }
+      const int nxt = e + 1;
+      if (nxt == W.b || ((W.cm >> nxt) & 1ull)) {  // chunk [c, nxt) complete
+        const uint32_t key = W.key_at(c);
+        if (key != bad_key) {
+          const int writer = turn % RPI;
+          int64_t slot = 0;
+          const bool whole = chunk_is_whole_run(W, c, nxt, N, lane == 0, &slot, mc_len, mc_list, mc_count);
+          if (grp == writer) {
+            float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
+            if (whole) {
+#pragma unroll
+              for (int k = 0; k < CPLN; k += 4) red_add4(dst + k, acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < CPLN; k += 4)
+                *reinterpret_cast<float4*>(dst + k) = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+            }
+          }
+          ++turn;
+        }
+      }
+    }
+    __syncwarp();  // the next batch reuses the staging buffer
+  }
+}
+
+// Generic fold for row sizes the wide fold does not cover: lanes own
+// columns l, l+32, ... of every row; one warp-wide load per hit.
+template <bool BF16>
+__global__ void __launch_bounds__(kFoldThreads, 3)
+fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
+                    const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
+                    int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
+  constexpr int kBatch = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5;
+  if (w * 32 >= N) return;
+  Window W;
+  if (!window_setup(K, I, N, w, W)) return;
+  Cols<0> acc;
+#pragma unroll
+  for (int k = 0; k < Cols<0>::n; ++k) acc.v[k] = 0.f;
+  int c = W.a;
+  for (int e0 = W.a; e0 < W.b; e0 += kBatch) {
+    Cols<0> g[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
       const int e = e0 + u;
-      if (e < b) {
-        const uint32_t idx = e < 32 ? __shfl_sync(kFull, iA, e) : __shfl_sync(kFull, iB, e - 32);
-        load_cols<CPL, BF16>(grad, idx, D, g[u]);
+      if (e < W.b) {
+        const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
+        load_cols<0, BF16>(grad, e < 32 ? ia : ib, D, g[u]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kFoldBatch; ++u) {
+    for (int u = 0; u < kBatch; ++u) {
       const int e = e0 + u;
-      if (e < b) {
-        if ((cm >> e) & 1ull) {
+      if (e < W.b) {
+        if ((W.cm >> e) & 1ull) {
           c = e;
 #pragma unroll
-          for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = g[u].v[k];
+          for (int k = 0; k < Cols<0>::n; ++k) acc.v[k] = g[u].v[k];
         } else {
 #pragma unroll
-          for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = acc.v[k] + g[u].v[k];
+          for (int k = 0; k < Cols<0>::n; ++k) acc.v[k] = acc.v[k] + g[u].v[k];
         }
         const int nxt = e + 1;
-        const bool chunk_end = nxt == b || ((cm >> nxt) & 1ull);
-        if (chunk_end) {
-          const uint32_t key = c < 32 ? __shfl_sync(kFull, kA, c) : __shfl_sync(kFull, kB, c - 32);
+        if (nxt == W.b || ((W.cm >> nxt) & 1ull)) {
+          const uint32_t key = W.key_at(c);
           if (key != bad_key) {
-            const bool is_head = (hm >> c) & 1ull;
-            const bool run_ends = (p0 + nxt >= N) || ((hm >> nxt) & 1ull);
-            if (is_head && run_ends) {
-              red_add_row<CPL>(table_grad, key, D, acc);
-            } else {
-              const int64_t pos = p0 + c;
-              store_slot<CPL>(csum, 2 * (pos >> 5) + (is_head ? 1 : 0), D, acc);
-              if (lane == 0) {
-                if (is_head) mc_list[atomicAdd(mc_count, 1)] = static_cast<int>(pos);
-                if (run_ends) {
-                  const int64_t s = run_start(c);
-                  mc_len[s >> 5] = static_cast<int>(p0 + nxt - s);
-                }
-              }
-            }
+            int64_t slot = 0;
+            if (chunk_is_whole_run(W, c, nxt, N, lane == 0, &slot, mc_len, mc_list, mc_count))
+              red_add_row<0>(table_grad, key, D, acc);
+            else
+              store_slot<0>(csum, slot, D, acc);
           }
         }
       }
@@ -452,7 +674,7 @@ fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, c
     const int nc = static_cast<int>((len + kChunk - 1) / kChunk);
     const uint32_t key = K[c0];
     if (key >= bad_key) continue;
-    Cols<CPL> acc, x;
+    Cols<CPL> acc;
     auto load_slot = [&](int64_t slot, Cols<CPL>& y) {
       if constexpr (CPL == 0) {
 #pragma unroll
@@ -465,10 +687,18 @@ fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, c
       }
     };
     load_slot(2 * (c0 >> 5) + 1, acc);
-    for (int m = 1; m < nc; ++m) {
-      load_slot(2 * ((c0 + static_cast<int64_t>(m) * kChunk) >> 5), x);
+    constexpr int kAhead = 8;  // chunk sums loaded ahead of the in-order adds
+    for (int m0 = 1; m0 < nc; m0 += kAhead) {
+      Cols<CPL> y[kAhead];
 #pragma unroll
-      for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = acc.v[k] + x.v[k];
+      for (int u = 0; u < kAhead; ++u)
+        if (m0 + u < nc) load_slot(2 * ((c0 + static_cast<int64_t>(m0 + u) * kChunk) >> 5), y[u]);
+#pragma unroll
+      for (int u = 0; u < kAhead; ++u)
+        if (m0 + u < nc) {
+#pragma unroll
+          for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = acc.v[k] + y[u].v[k];
+        }
     }
     red_add_row<CPL>(table_grad, key, D, acc);
   }
@@ -498,8 +728,9 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
 // host side
 // ---------------------------------------------------------------------------
 struct Layout {
-  size_t keys[2], vals[2], hist, csum, mc_len, mc_list, mc_count, total;
-  int num_tiles;
+  size_t keys[2], vals[2], hist, gtot, csum, mc_len, mc_list, zeroed, total;
+  size_t zeroed_bytes;  // tickets of every pass + the heavy-run counter, cleared per call
+  int num_tiles, num_groups, max_passes;
   int64_t nwin;
 };
 
@@ -508,6 +739,8 @@ size_t align_up(size_t x) { return (x + 255) & ~size_t{255}; }
 Layout layout_for(int64_t N, int D) {
   Layout L{};
   L.num_tiles = static_cast<int>((N + kSortTile - 1) / kSortTile);
+  L.num_groups = (L.num_tiles + kTilesPerGroup - 1) / kTilesPerGroup;
+  L.max_passes = 4;
   L.nwin = (N + 31) / 32;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -518,10 +751,12 @@ Layout layout_for(int64_t N, int D) {
   for (int b = 0; b < 2; ++b) L.keys[b] = take(sizeof(uint32_t) * N);
   for (int b = 0; b < 2; ++b) L.vals[b] = take(sizeof(uint32_t) * N);
   L.hist = take(sizeof(uint32_t) * kRadix * static_cast<size_t>(L.num_tiles));
+  L.gtot = take(sizeof(uint32_t) * kRadix * static_cast<size_t>(L.num_groups));
   L.csum = take(sizeof(float) * 2 * static_cast<size_t>(L.nwin) * D);
   L.mc_len = take(sizeof(int) * L.nwin);
   L.mc_list = take(sizeof(int) * L.nwin);
-  L.mc_count = take(sizeof(int));
+  L.zeroed_bytes = sizeof(unsigned int) * (static_cast<size_t>(L.max_passes) * (L.num_groups + 1) + 1);
+  L.zeroed = take(L.zeroed_bytes);
   L.total = off;
   return L;
 }
@@ -545,7 +780,6 @@ ple_status_t check_grad_args(const ple_plan_t* plan, const int64_t* rows, int64_
   return PLE_OK;
 }
 
-bool g_scatter_smem_set[64];
 
 }  // namespace
 }  // namespace ple
@@ -572,45 +806,39 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   cudaError_t e;
   unsigned int* status = status_word(&e);
   if (status == nullptr) return cuda_fail(e);
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !g_scatter_smem_set[dev]) {
-    e = cudaFuncSetAttribute(scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kScatterSmem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(scatter_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kScatterSmem));
-    if (e != cudaSuccess) return cuda_fail(e);
-    g_scatter_smem_set[dev] = true;
-  }
   auto* ws = static_cast<unsigned char*>(workspace);
   uint32_t* keys[2] = {reinterpret_cast<uint32_t*>(ws + L.keys[0]), reinterpret_cast<uint32_t*>(ws + L.keys[1])};
   uint32_t* vals[2] = {reinterpret_cast<uint32_t*>(ws + L.vals[0]), reinterpret_cast<uint32_t*>(ws + L.vals[1])};
   uint32_t* hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+  uint32_t* gtot = reinterpret_cast<uint32_t*>(ws + L.gtot);
   float* csum = reinterpret_cast<float*>(ws + L.csum);
   int* mc_len = reinterpret_cast<int*>(ws + L.mc_len);
   int* mc_list = reinterpret_cast<int*>(ws + L.mc_list);
-  int* mc_count = reinterpret_cast<int*>(ws + L.mc_count);
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(ws + L.zeroed);
+  int* mc_count = reinterpret_cast<int*>(tickets + static_cast<size_t>(L.max_passes) * (L.num_groups + 1));
   const auto s = static_cast<cudaStream_t>(stream);
 
   // key bits: keys lie in [0, num_rows] (num_rows marks a bad row)
   int bits = 0;
   while (bits < 32 && (static_cast<uint64_t>(plan->num_rows) >> bits) != 0) ++bits;
   const int passes = (bits + 7) / 8;
-  const int M = kRadix * L.num_tiles;
 
-  keys_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(rows, N, plan->num_rows, keys[0], hist, L.num_tiles, mc_count,
-                                                   status);
+  e = cudaMemsetAsync(tickets, 0, L.zeroed_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  keys_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(rows, N, plan->num_rows, keys[0], hist, gtot, tickets,
+                                                   L.num_tiles, status);
   int cur = 0;
   for (int p = 0; p < passes; ++p) {
-    if (p > 0) hist_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], N, 8 * p, hist, L.num_tiles);
-    scan_kernel<<<1, kScanThreads, 0, s>>>(hist, M);
+    if (p > 0)
+      hist_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], N, 8 * p, hist, gtot,
+                                                       tickets + static_cast<size_t>(p) * (L.num_groups + 1),
+                                                       L.num_tiles);
     if (p == 0)
-      scatter_kernel<true><<<L.num_tiles, kSortThreads, kScatterSmem, s>>>(keys[cur], nullptr, keys[1 - cur],
-                                                                          vals[1 - cur], hist, N, 0, L.num_tiles);
+      scatter_kernel<true><<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], nullptr, keys[1 - cur], vals[1 - cur],
+                                                                hist, gtot, N, 0, L.num_tiles);
     else
-      scatter_kernel<false><<<L.num_tiles, kSortThreads, kScatterSmem, s>>>(
-          keys[cur], vals[cur], keys[1 - cur], vals[1 - cur], hist, N, 8 * p, L.num_tiles);
+      scatter_kernel<false><<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], vals[cur], keys[1 - cur],
+                                                                 vals[1 - cur], hist, gtot, N, 8 * p, L.num_tiles);
     cur = 1 - cur;
   }
   const uint32_t* Ks = keys[cur];
@@ -618,27 +846,43 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   const uint32_t bad_key = static_cast<uint32_t>(plan->num_rows);
   const unsigned fold_blocks = static_cast<unsigned>((L.nwin * 32 + kFoldThreads - 1) / kFoldThreads);
   const unsigned heavy_blocks = static_cast<unsigned>(sm_count() * 4);
-  const int cpl = cols_per_lane(D);
   const bool bf = gdt == PLE_BF16;
-#define PLE_FOLD(CPL)                                                                                      \
-  do {                                                                                                     \
-    if (bf)                                                                                                \
-      fold_kernel<CPL, true><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad, \
-                                                                  csum, mc_len, mc_list, mc_count);        \
-    else                                                                                                   \
-      fold_kernel<CPL, false><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad, \
-                                                                   csum, mc_len, mc_list, mc_count);       \
-    fold_heavy_kernel<CPL><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list,     \
-                                                                 mc_count, D, table_grad);                 \
-  } while (0)
-  switch (cpl) {
-    case 1: PLE_FOLD(1); break;
-    case 2: PLE_FOLD(2); break;
-    case 4: PLE_FOLD(4); break;
-    case 8: PLE_FOLD(8); break;
-    default: PLE_FOLD(0); break;
+  const int lanes_per_row = static_cast<int>(static_cast<int64_t>(D) * (bf ? 2 : 4) / 16);
+  const unsigned wide_blocks = static_cast<unsigned>((L.nwin + kWideWarps - 1) / kWideWarps);
+#define PLE_FOLD_WIDE(LW)                                                                                   \
+  case LW:                                                                                                  \
+    if (bf)                                                                                                 \
+      fold_wide_kernel<LW, true><<<wide_blocks, kWideWarps * 32, 0, s>>>(Ks, Is, N, bad_key, grad, D,       \
+                                                                         table_grad, csum, mc_len, mc_list, \
+                                                                         mc_count);                         \
+    else                                                                                                    \
+      fold_wide_kernel<LW, false><<<wide_blocks, kWideWarps * 32, 0, s>>>(Ks, Is, N, bad_key, grad, D,      \
+                                                                          table_grad, csum, mc_len, mc_list, \
+                                                                          mc_count);                        \
+    break;
+  switch (lanes_per_row) {
+    PLE_FOLD_WIDE(1)
+    PLE_FOLD_WIDE(2)
+    PLE_FOLD_WIDE(4)
+    PLE_FOLD_WIDE(8)
+    PLE_FOLD_WIDE(16)
+    PLE_FOLD_WIDE(32)
+    default:
+      if (bf)
+        fold_generic_kernel<true><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad,
+                                                                       csum, mc_len, mc_list, mc_count);
+      else
+        fold_generic_kernel<false><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad,
+                                                                        csum, mc_len, mc_list, mc_count);
   }
-#undef PLE_FOLD
+#undef PLE_FOLD_WIDE
+  switch (cols_per_lane(D)) {
+    case 1: fold_heavy_kernel<1><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+    case 2: fold_heavy_kernel<2><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+    case 4: fold_heavy_kernel<4><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+    case 8: fold_heavy_kernel<8><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+    default: fold_heavy_kernel<0><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+  }
   return check_launch();
 }
 

@@ -110,19 +110,21 @@ hash_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
 }
 
 // ---------------------------------------------------------------------------
-// Row streaming shared by the fused lookup and the gather.
+// Row streaming shared by the fused lookup and the gather: `lanes` threads
+// (a warp or a block) copy nhits rows, vector q of the output being column
+// q mod V of hit q div V.
 // ---------------------------------------------------------------------------
-template <int VL>
+template <int VL, int kLanes>
 __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ table,
                                           const int64_t* __restrict__ rowoff, int nhits, int v_rt,
-                                          unsigned char* __restrict__ out) {
+                                          unsigned char* __restrict__ out, int tid) {
   const int V = VL >= 0 ? (1 << VL) : v_rt;
   const int total = nhits * V;
-  for (int base = threadIdx.x; base < total; base += kBlock * kUnroll) {
+  for (int base = tid; base < total; base += kLanes * kUnroll) {
     uint4 v[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int q = base + u * kBlock;
+      const int q = base + u * kLanes;
       if (q < total) {
         const int hit = VL >= 0 ? (q >> VL) : q / V;
         const int col = q - hit * V;
@@ -132,48 +134,52 @@ __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ tabl
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int q = base + u * kBlock;
+      const int q = base + u * kLanes;
       if (q < total) st_cs(out + static_cast<int64_t>(q) * 16, v[u]);
     }
   }
 }
 
-// Fused lookup: TT tokens per block.  Warp 0 hashes the tile's tokens, all
-// threads turn the order hashes into rows (one remainder per hit), then the
-// block streams the tile's TT*H rows.
-template <int TT, int VL>
+// Fused lookup.  Every warp owns TW consecutive tokens and works alone (no
+// block barrier after the constants are staged): its first TW lanes hash the
+// tokens, the warp turns the order hashes into TW*H row offsets in its own
+// slice of shared memory, then streams those rows.  Warps drift apart, so one
+// warp's hashing overlaps other warps' copies.
+template <int TW, int VL>
 __global__ void __launch_bounds__(kBlock, 4)
 lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
               const int32_t* __restrict__ cu, int32_t num_seqs, const unsigned char* __restrict__ table,
               int64_t num_rows, int32_t row_bytes, unsigned char* __restrict__ out,
               int64_t* __restrict__ rows_out, unsigned int* status) {
-  static_assert(TT <= 32, "one warp hashes the tile");
+  static_assert(TW <= 32, "the first TW lanes hash the warp's tokens");
   extern __shared__ __align__(16) unsigned char smem[];
   const int H = hp.num_heads;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   HeadConst* consts = reinterpret_cast<HeadConst*>(smem);
-  int64_t* hsh = reinterpret_cast<int64_t*>(consts + H);   // [TT][kMaxOrder-1]
-  int64_t* rowoff = hsh + TT * (kMaxOrder - 1);            // [TT*H]
+  int64_t* hsh = reinterpret_cast<int64_t*>(consts + H) + warp * TW * (kMaxOrder - 1);  // [TW][7]
+  int64_t* rowoff = reinterpret_cast<int64_t*>(consts + H) + (kBlock / 32) * TW * (kMaxOrder - 1) +
+                    warp * TW * H;                                                        // [TW*H]
   load_consts(hp, consts);
   check_seqlens(cu, num_seqs, T, status);
+  __syncthreads();
 
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * TT;
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + warp) * TW;
+  if (t0 >= T) return;
+  {
     const int64_t t = t0 + lane;
-    const bool valid = lane < TT && t < T;
+    const bool valid = lane < TW && t < T;
     int64_t hs[kMaxOrder - 1];
     order_hashes(hp, tokens, cu, num_seqs, t, valid, hs);
-    if (lane < TT) {
+    if (lane < TW) {
 #pragma unroll
       for (int m = 0; m < kMaxOrder - 1; ++m) hsh[lane * (kMaxOrder - 1) + m] = hs[m];
     }
   }
-  __syncthreads();
-
-  const int ntok = static_cast<int>(min(static_cast<int64_t>(TT), T - t0));
+  __syncwarp();
+  const int ntok = static_cast<int>(min(static_cast<int64_t>(TW), T - t0));
   const int nhits = ntok * H;
   const int G = hp.heads_per_ngram;
-  for (int q = threadIdx.x; q < nhits; q += kBlock) {
+  for (int q = lane; q < nhits; q += 32) {
     const int tl = q / H;
     const int j = q - tl * H;
     const HeadConst c = consts[j];
@@ -182,8 +188,8 @@ lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T
     rowoff[q] = row < num_rows ? row * row_bytes : -1;
     if (rows_out != nullptr) rows_out[t0 * H + q] = row;
   }
-  __syncthreads();
-  copy_hits<VL>(table, rowoff, nhits, row_bytes >> 4, out + t0 * H * row_bytes);
+  __syncwarp();
+  copy_hits<VL, 32>(table, rowoff, nhits, row_bytes >> 4, out + t0 * H * row_bytes, lane);
 }
 
 constexpr int kGatherHits = 512;  // hits per block of the plain gather
@@ -205,7 +211,7 @@ gather_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows,
   }
   if (bad) raise_flag(status, PLE_ERR_BAD_ROW);
   __syncthreads();
-  copy_hits<VL>(table, rowoff, nh, row_bytes >> 4, out + h0 * row_bytes);
+  copy_hits<VL, kBlock>(table, rowoff, nh, row_bytes >> 4, out + h0 * row_bytes, threadIdx.x);
 }
 
 int log2_exact(int v) {
@@ -214,22 +220,25 @@ int log2_exact(int v) {
   return -1;
 }
 
-template <int TT>
+template <int TW>
 ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
                            int32_t S, const void* table, void* out, int64_t* rows_out, unsigned int* status,
                            cudaStream_t stream) {
   const int H = plan->hp.num_heads;
-  const size_t smem = H * sizeof(HeadConst) + TT * (kMaxOrder - 1) * sizeof(int64_t) +
-                      static_cast<size_t>(TT) * H * sizeof(int64_t);
-  const dim3 grid(static_cast<unsigned>((T + TT - 1) / TT));
+  constexpr int kWarps = kBlock / 32;
+  const size_t smem = H * sizeof(HeadConst) + kWarps * TW * (kMaxOrder - 1) * sizeof(int64_t) +
+                      static_cast<size_t>(kWarps) * TW * H * sizeof(int64_t);
+  if (smem > 48 * 1024) return PLE_ERR_UNSUPPORTED;  // not reached: TW*H <= 512 keeps it under 48 KB
+  const int64_t warps = (T + TW - 1) / TW;
+  const dim3 grid(static_cast<unsigned>((warps + kWarps - 1) / kWarps));
   const auto* tb = static_cast<const unsigned char*>(table);
   auto* ob = static_cast<unsigned char*>(out);
   const int rb = plan->row_bytes;
   const int64_t R = plan->num_rows;
-#define PLE_LOOKUP_CASE(VL)                                                                           \
-  case VL:                                                                                            \
-    lookup_kernel<TT, VL><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,     \
-                                                          rows_out, status);                                     \
+#define PLE_LOOKUP_CASE(VL)                                                                            \
+  case VL:                                                                                             \
+    lookup_kernel<TW, VL><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,     \
+                                                          rows_out, status);                           \
     break;
   switch (log2_exact(rb >> 4)) {
     PLE_LOOKUP_CASE(0)
@@ -240,7 +249,7 @@ ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_
     PLE_LOOKUP_CASE(5)
     PLE_LOOKUP_CASE(6)
     default:
-      lookup_kernel<TT, -1><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
+      lookup_kernel<TW, -1><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
                                                             rows_out, status);
   }
 #undef PLE_LOOKUP_CASE
@@ -298,11 +307,21 @@ ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T
   cudaError_t e;
   unsigned int* status = status_word(&e);
   if (status == nullptr) return cuda_fail(e);
-  const int64_t tiles32 = (T + 31) / 32;
   const auto s = static_cast<cudaStream_t>(stream);
-  if (tiles32 >= 8LL * sm_count())
-    return launch_lookup<32>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-  return launch_lookup<16>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+  // tokens per warp: about 1-4K 16-byte vectors of copy work per warp, but
+  // enough warps to fill every SM several times over
+  const int64_t vec_per_token = static_cast<int64_t>(plan->hp.num_heads) * (plan->row_bytes >> 4);
+  int tw = 32;
+  while (tw > 4 && (tw * vec_per_token > 4096 || (T + tw - 1) / tw < 32LL * sm_count())) tw >>= 1;
+  while (tw > 1 && tw * plan->hp.num_heads > 512) tw >>= 1;  // row offsets of 8 warps stay <= 32 KB
+  switch (tw) {
+    case 32: return launch_lookup<32>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    case 16: return launch_lookup<16>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    case 8: return launch_lookup<8>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    case 4: return launch_lookup<4>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    case 2: return launch_lookup<2>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    default: return launch_lookup<1>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+  }
 }
 
 ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* table, void* out,

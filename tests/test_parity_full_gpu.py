@@ -105,7 +105,7 @@ def test_backward_stress_full(cuda_device):
     ref_rows = _oracle_rows(w)
     np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
     # heavy repetition: the hottest row is hit thousands of times
-    counts = np.bincount(np.unique(ref_rows, return_inverse=True)[1])
+    counts = np.bincount(np.unique(ref_rows.ravel(), return_inverse=True)[1].ravel())
     assert counts.max() > 1000
     check_backward_full(w, cuda_device, ref_rows)
 
