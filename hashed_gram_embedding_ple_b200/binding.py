@@ -31,7 +31,8 @@ _DTYPES = {torch.float32: PLE_F32, torch.bfloat16: PLE_BF16}
 
 # every symbol include/ple.h declares
 EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_gather",
-           "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic", "ple_status",
+           "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic",
+           "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_status",
            "ple_strerror", "ple_last_cuda_error")
 
 
@@ -74,12 +75,16 @@ def _lib():
         lib.ple_grad_scatter_workspace_bytes.restype = sz
         lib.ple_grad_scatter.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
         lib.ple_grad_scatter_atomic.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
+        lib.ple_grad_scatter_noalloc.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
+        lib.ple_grad_scatter_noalloc_scratch_bytes.argtypes = []
+        lib.ple_grad_scatter_noalloc_scratch_bytes.restype = sz
         lib.ple_status.argtypes = [vp]
         lib.ple_strerror.argtypes = [ctypes.c_int]
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
         for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_gather", "ple_grad_scatter",
-                     "ple_grad_scatter_atomic", "ple_status", "ple_last_cuda_error"):
+                     "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_status",
+                     "ple_last_cuda_error"):
             getattr(lib, name).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -232,6 +237,26 @@ def ple_grad_scatter_atomic(plan: Plan, rows, grad_out, table_grad):
     _check(_lib().ple_grad_scatter_atomic(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
                                           _stream(rows.device)), "ple_grad_scatter_atomic")
     return table_grad
+
+
+def ple_grad_scatter_noalloc(plan: Plan, rows, grad_out, table_grad):
+    """Deterministic gradient using the library's fixed scratch area (no
+    workspace, no allocation); see include/ple.h for the size limit and the
+    rules on overlapping calls."""
+    _as_i64(rows, "rows")
+    gdt = _grad_dtype(grad_out)
+    if table_grad.dtype != torch.float32 or not table_grad.is_contiguous():
+        raise ValueError("table_grad must be contiguous float32")
+    N = rows.numel()
+    if grad_out.numel() != N * plan.head_dim:
+        raise ValueError("grad_out must hold num_hits * head_dim values")
+    _check(_lib().ple_grad_scatter_noalloc(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
+                                           _stream(rows.device)), "ple_grad_scatter_noalloc")
+    return table_grad
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_lib().ple_grad_scatter_noalloc_scratch_bytes())
 
 
 def ple_status(device=None) -> int:

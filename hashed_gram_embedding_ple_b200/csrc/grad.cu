@@ -24,6 +24,8 @@
 //      sums in order and adds the result into table_grad.
 // The final add is a vector fp32 reduction (red.global.add) issued by the one
 // warp that owns the row, so it is the single add table_grad + S_r.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace ple {
@@ -917,5 +919,53 @@ ple_status_t ple_grad_scatter_atomic(const ple_plan_t* plan, const int64_t* rows
 #undef PLE_ATOMIC
   return check_launch();
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Gradient scatter without any allocation by anyone.
+//
+// Some callers cannot hand the library a workspace: a serving process whose
+// device memory is reserved up front and may not grow while requests run, a
+// host plugin that is not allowed to call the CUDA allocator, or a hot loop
+// where cudaMalloc could synchronise the device and stall every stream.  For
+// them the library keeps one fixed scratch area
+// of kNoAllocScratchBytes in device memory (allocated with the module, held by
+// every GPU that loads the library until the process exits) and runs the same
+// deterministic sort-and-fold kernels in it.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t{32} << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, one per device.  In host code the
+// array's name only stands in for the symbol; its device address has to be
+// looked up with that device current.
+std::atomic<void*> g_noalloc_addr[64];
+
+}  // namespace
+
+extern "C" {
+
+ple_status_t ple_grad_scatter_noalloc(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* grad,
+                                      ple_dtype_t gdt, float* table_grad, void* stream) {
+  if (plan == nullptr || N < 0) return PLE_ERR_INVALID_ARG;
+  if (N == 0) return check_grad_args(plan, rows, N, grad, gdt, table_grad);
+  if (ple_grad_scatter_workspace_bytes(plan, N) > kNoAllocScratchBytes) return PLE_ERR_WORKSPACE;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return PLE_ERR_UNSUPPORTED;
+  void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {  // first call on this device: look the address up
+    e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_addr[dev].store(scratch, std::memory_order_release);
+  }
+  return ple_grad_scatter(plan, rows, N, grad, gdt, table_grad, scratch, kNoAllocScratchBytes, stream);
+}
+
+size_t ple_grad_scatter_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 }  // extern "C"

@@ -143,6 +143,29 @@ ple_status_t ple_grad_scatter_atomic(const ple_plan_t* plan, const int64_t* rows
                                      const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,
                                      void* stream);
 
+/* The same deterministic gradient as ple_grad_scatter, for callers that
+ * cannot provide a workspace: serving processes whose device memory is
+ * reserved up front and may not grow while requests run, plugin hosts that
+ * forbid calls to the CUDA allocator, or hot loops where cudaMalloc could
+ * synchronise the device.  No counterpart on the source pages: it is a service
+ * of this library.  Nothing is allocated by anyone: the kernels use a fixed
+ * scratch area of ple_grad_scatter_noalloc_scratch_bytes() (32 MiB) that the
+ * library holds in the device memory of every GPU that loads it, until the
+ * process exits.  Sizes whose workspace (ple_grad_scatter_workspace_bytes)
+ * exceeds that area are rejected with PLE_ERR_WORKSPACE before anything is
+ * launched; use ple_grad_scatter with a caller workspace for them.  The first
+ * call on a device looks up the scratch area's device address (make that
+ * first call before any stream capture).  All calls share the one area, so
+ * calls that overlap on the GPU (other streams, other host threads) race and
+ * must be serialised by the caller; each call clears what must start at zero.
+ * Other arguments, errors and results as ple_grad_scatter. */
+ple_status_t ple_grad_scatter_noalloc(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits,
+                                      const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,
+                                      void* stream);
+
+/* Bytes of the fixed scratch area ple_grad_scatter_noalloc works in. */
+size_t ple_grad_scatter_noalloc_scratch_bytes(void);
+
 /* Synchronise `stream`, then return and clear the async status word of the
  * current device (PLE_OK if no kernel flagged anything; otherwise the
  * lowest-numbered flagged error).  The word is shared by all plans and
