@@ -346,7 +346,7 @@ def main():
             roofline = bwd_roof
 
     passes = math.ceil(max(1, int(w.num_rows).bit_length()) / 8)
-    launches_per_step = 1 + ((3 * passes + 2) if do_bwd else 0)
+    launches_per_step = 1 + ((2 * passes + 2) if do_bwd else 0)  # lookup; keys, passes x scatter, passes-1 x hist, two folds
     value = world * T / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers

@@ -23,6 +23,7 @@ PLE_ERR_WORKSPACE = 4
 PLE_ERR_CUDA = 5
 PLE_ERR_BAD_ROW = 6
 PLE_ERR_BAD_SEQLENS = 7
+PLE_ERR_TIMEOUT = 8
 
 PLE_F32 = 0
 PLE_BF16 = 1

@@ -83,6 +83,31 @@ __device__ __forceinline__ int32_t find_sequence(const int32_t* __restrict__ cu,
   return lo;
 }
 
+// Programmatic dependent launch (sm_90+).  A kernel launched with
+// launch_after() may start while its predecessor in the stream is still
+// draining; it must call wait_for_prior_grid() before it touches anything the
+// predecessor writes (the hardware releases the wait once the predecessor has
+// completed and its memory is visible).  allow_next_grid() lets the next
+// grid be scheduled early.
+__device__ __forceinline__ void wait_for_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_after(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 }  // namespace ple
 
 // ---------------------------------------------------------------------------

@@ -24,6 +24,7 @@
 //      sums in order and adds the result into table_grad.
 // The final add is a vector fp32 reduction (red.global.add) issued by the one
 // warp that owns the row, so it is the single add table_grad + S_r.
+#include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
@@ -32,11 +33,7 @@ namespace ple {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kSortThreads = 256;
-constexpr int kSortItems = 4;
-constexpr int kSortTile = kSortThreads * kSortItems;  // keys per sort tile
 constexpr int kRadix = 256;
-constexpr int kWarpsPerSortBlock = kSortThreads / 32;
 constexpr int kChunk = 32;
 constexpr uint32_t kNoKey = 0xffffffffu;  // past the end; never a real key
 constexpr int kFoldThreads = 256;
@@ -48,217 +45,243 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // ---------------------------------------------------------------------------
-// radix sort
+// radix sort: one cooperative kernel runs every pass
 //
-// Tiles of 4096 keys; inside a tile warp w owns positions [512w, 512w+512),
-// read in 16 rounds of 32, so (warp, round, lane) is the tile order.
-// Histograms are stored tile-major, hist[tile][digit].  Tiles form groups of
-// 32: the last block of a group to finish its histogram (atomic ticket, no
-// waiting) turns the group's histograms into in-group exclusive prefixes and
-// writes the group's digit totals.  A scatter block then derives its global
-// digit offsets from the (few) group totals itself, so no device-wide scan
-// kernel is needed.
+// All blocks of the grid are resident at once (cooperative launch), so the
+// phases of a pass are separated by a grid barrier instead of kernel
+// boundaries.  Block b owns the contiguous positions [b*seg, (b+1)*seg) of
+// the pass's input.  Per pass (8-bit digit at `shift`):
+//   H: block histograms of its positions -> hist[b][digit];
+//   P: one block per digit scans hist[.][digit] over the blocks ->
+//      off[b][digit] (keys of that digit in earlier blocks) and total[digit];
+//   S: block b walks its positions in tiles of 2048 in order and writes each
+//      key to  digit_base + off[b][digit] + (same digit earlier in its
+//      positions), the last term from per-warp running counts: stable.
+// The barrier's wait is bounded: past the limit the block raises
+// PLE_ERR_TIMEOUT and leaves (the result is then unspecified, nothing hangs).
 // ---------------------------------------------------------------------------
-constexpr int kTilesPerGroup = 32;
+constexpr int kCoopThreads = 512;
+constexpr int kCoopWarps = kCoopThreads / 32;
+constexpr int kCoopItems = 4;
+constexpr int kCoopTile = kCoopThreads * kCoopItems;  // keys per tile of the scatter phase
+constexpr int kCoopMaxBlocks = 2 * kCoopThreads;      // the prefix phase scans <= 2 blocks per thread
+constexpr unsigned kSpinLimit = 1u << 22;             // a few seconds of polling, then give up
+
+// Lanes of the warp holding the same BITS-bit value as this lane (valid
+// lanes only): one ballot per bit, each lane keeping the lanes that agree
+// with it on that bit.
+template <int BITS>
+__device__ __forceinline__ unsigned peers_of(bool valid, uint32_t value) {
+  unsigned peers = __ballot_sync(kFull, valid);
+#pragma unroll
+  for (int bit = 0; bit < BITS; ++bit) {
+    const bool set = (value >> bit) & 1u;
+    const unsigned m = __ballot_sync(kFull, set);
+    peers &= set ? m : ~m;
+  }
+  return valid ? peers : 0u;
+}
 
 // Warp-aggregated shared-memory histogram update for one key per lane.
 __device__ __forceinline__ void hist_add(uint32_t* h, bool valid, uint32_t digit) {
-  const unsigned peers = __match_any_sync(kFull, valid ? digit : 0x100u);
+  const unsigned peers = peers_of<8>(valid, digit);
   if (valid && (peers & lanemask_lt()) == 0) atomicAdd(&h[digit], __popc(peers));
 }
 
-__device__ __forceinline__ int64_t tile_pos(int64_t tile, int warp, int r, int lane) {
-  return tile * kSortTile + warp * (kSortTile / kWarpsPerSortBlock) + r * 32 + lane;
-}
-
-// Block-wide exclusive sum over the 256 threads (one value per thread).
-__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t x, uint32_t* warp_tot) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// Block-wide exclusive sum (every thread passes one value); *total gets the sum.
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t x, uint32_t* warp_tot, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   uint32_t incl = x;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const uint32_t y = __shfl_up_sync(kFull, incl, d);
     if (lane >= d) incl += y;
   }
+  __syncthreads();  // warp_tot may still be read by a previous call
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
-  uint32_t before = 0;
-  for (int w = 0; w < warp; ++w) before += warp_tot[w];
+  uint32_t before = 0, all = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    const uint32_t t = warp_tot[w];
+    if (w < warp) before += t;
+    all += t;
+  }
+  *total = all;
   return before + incl - x;
 }
 
-// Publish this block's histogram.  The last block of a group of 32 tiles to
-// arrive (atomic ticket, nobody waits) turns the group's histograms into
-// in-group exclusive prefixes and writes the group's digit totals; the last
-// group to finish then turns the group totals into gbase[group][digit] =
-// (keys of smaller digits) + (keys of this digit in earlier groups).  A
-// scatter block's global offset for digit d is gbase[its group][d] +
-// hist[its tile][d].
-__device__ void publish_histogram(const uint32_t* h, uint32_t* __restrict__ hist, uint32_t* __restrict__ gtot,
-                                  unsigned int* __restrict__ tickets, int num_tiles) {
-  __shared__ bool is_last;
-  __shared__ uint32_t warp_tot[kWarpsPerSortBlock];
-  const int tile = blockIdx.x, d = threadIdx.x;
-  const int ngroups = (num_tiles + kTilesPerGroup - 1) / kTilesPerGroup;
-  unsigned int* group_done = tickets + ngroups;  // one more counter after the per-group tickets
-  hist[static_cast<int64_t>(tile) * kRadix + d] = h[d];
-  __threadfence();
-  __syncthreads();
-  const int g = tile / kTilesPerGroup;
-  const int first = g * kTilesPerGroup;
-  const int n = min(kTilesPerGroup, num_tiles - first);
-  if (threadIdx.x == 0) is_last = atomicAdd(&tickets[g], 1u) == static_cast<unsigned>(n - 1);
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  {
-    uint32_t v[kTilesPerGroup];
-    uint32_t* col = hist + static_cast<int64_t>(first) * kRadix + d;
-#pragma unroll
-    for (int k = 0; k < kTilesPerGroup; ++k) v[k] = k < n ? __ldcg(col + k * kRadix) : 0;  // all loads first
-    uint32_t run = 0;
-#pragma unroll
-    for (int k = 0; k < kTilesPerGroup; ++k) {
-      if (k < n) col[k * kRadix] = run;
-      run += v[k];
-    }
-    gtot[static_cast<int64_t>(g) * kRadix + d] = run;
-  }
-  __threadfence();
+// Grid barrier for a cooperative grid.  The counter only grows within a call
+// (it is cleared before the launch); each arrival waits for the next multiple
+// of the grid size.
+__device__ bool grid_barrier(unsigned int* bar, unsigned int* status) {
+  __shared__ bool ok;
   __syncthreads();
   if (threadIdx.x == 0) {
-    tickets[g] = 0;  // ready for the next pass / call
-    is_last = atomicAdd(group_done, 1u) == static_cast<unsigned>(ngroups - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  // exclusive prefix over groups per digit, then the digit base over digits
-  uint32_t total = 0;
-#pragma unroll 8
-  for (int k = 0; k < ngroups; ++k) total += __ldcg(gtot + static_cast<int64_t>(k) * kRadix + d);
-  const uint32_t digit_base = block_exclusive_sum(total, warp_tot);
-  uint32_t run = digit_base;
-  for (int k0 = 0; k0 < ngroups; k0 += 8) {
-    uint32_t v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = k0 + k < ngroups ? __ldcg(gtot + static_cast<int64_t>(k0 + k) * kRadix + d) : 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (k0 + k < ngroups) gtot[static_cast<int64_t>(k0 + k) * kRadix + d] = run;
-      run += v[k];
-    }
-  }
-  if (threadIdx.x == 0) *group_done = 0;
-}
-
-__global__ void __launch_bounds__(kSortThreads)
-keys_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, uint32_t* __restrict__ keys,
-            uint32_t* __restrict__ hist, uint32_t* __restrict__ gtot, unsigned int* __restrict__ tickets,
-            int num_tiles, unsigned int* status) {
-  __shared__ uint32_t h[kRadix];
-  h[threadIdx.x] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  bool bad = false;
-#pragma unroll 4
-  for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = tile_pos(blockIdx.x, warp, r, lane);
-    const bool valid = i < N;
-    uint32_t key = 0;
-    if (valid) {
-      const int64_t v = rows[i];
-      const bool ok = v >= 0 && v < num_rows;
-      bad |= !ok;
-      key = ok ? static_cast<uint32_t>(v) : static_cast<uint32_t>(num_rows);
-      keys[i] = key;
-    }
-    hist_add(h, valid, key & (kRadix - 1));
-  }
-  if (bad) raise_flag(status, PLE_ERR_BAD_ROW);
-  __syncthreads();
-  publish_histogram(h, hist, gtot, tickets, num_tiles);
-}
-
-__global__ void __launch_bounds__(kSortThreads)
-hist_kernel(const uint32_t* __restrict__ keys, int64_t N, int shift, uint32_t* __restrict__ hist,
-            uint32_t* __restrict__ gtot, unsigned int* __restrict__ tickets, int num_tiles) {
-  __shared__ uint32_t h[kRadix];
-  h[threadIdx.x] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t key[kSortItems];
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = tile_pos(blockIdx.x, warp, r, lane);
-    key[r] = i < N ? keys[i] : 0;
-  }
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r)
-    hist_add(h, tile_pos(blockIdx.x, warp, r, lane) < N, (key[r] >> shift) & (kRadix - 1));
-  __syncthreads();
-  publish_histogram(h, hist, gtot, tickets, num_tiles);
-}
-
-// Stable rank-and-scatter of one tile.  Rank of a key = its tile's global
-// digit offset + the keys of that digit in earlier warps of the tile + the
-// keys of that digit earlier in its own warp (running per-warp counts,
-// updated round by round after every lane has read them).
-template <bool kIdentityVals>
-__global__ void __launch_bounds__(kSortThreads)
-scatter_kernel(const uint32_t* __restrict__ kin, const uint32_t* __restrict__ vin, uint32_t* __restrict__ kout,
-               uint32_t* __restrict__ vout, const uint32_t* __restrict__ hist, const uint32_t* __restrict__ gtot,
-               int64_t N, int shift, int num_tiles) {
-  __shared__ uint32_t wh[kWarpsPerSortBlock][kRadix];
-  __shared__ uint32_t tile_base[kRadix];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, d = threadIdx.x;
-  const int tile = blockIdx.x;
-  const int g = tile / kTilesPerGroup;
-
-  uint32_t key[kSortItems], val[kSortItems];
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    const int64_t i = tile_pos(tile, warp, r, lane);
-    key[r] = i < N ? kin[i] : kNoKey;
-    val[r] = i < N ? (kIdentityVals ? static_cast<uint32_t>(i) : vin[i]) : 0;
-  }
-  tile_base[d] = gtot[static_cast<int64_t>(g) * kRadix + d] + hist[static_cast<int64_t>(tile) * kRadix + d];
-#pragma unroll
-  for (int w = 0; w < kWarpsPerSortBlock; ++w) wh[w][d] = 0;
-  __syncthreads();
-  uint16_t rank[kSortItems];
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    const bool valid = tile_pos(tile, warp, r, lane) < N;
-    const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-    const unsigned peers = __match_any_sync(kFull, valid ? digit : 0x100u);
-    const unsigned lower = __popc(peers & lanemask_lt());
-    rank[r] = valid ? static_cast<uint16_t>(wh[warp][digit] + lower) : 0;
-    __syncwarp();
-    if (valid && lower == 0) wh[warp][digit] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  {
-    uint32_t run = 0;
-#pragma unroll
-    for (int w = 0; w < kWarpsPerSortBlock; ++w) {
-      const uint32_t c = wh[w][d];
-      wh[w][d] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
-    if (tile_pos(tile, warp, r, lane) < N) {
-      const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-      const uint32_t dst = tile_base[digit] + wh[warp][digit] + rank[r];
-      if (dst < N) {  // always true when the counts are consistent
-        kout[dst] = key[r];
-        vout[dst] = val[r];
+    __threadfence();
+    const unsigned int nblocks = gridDim.x;
+    const unsigned int old = atomicAdd(bar, 1u);
+    const unsigned int target = (old / nblocks + 1) * nblocks;
+    bool good = true;
+    for (unsigned int spins = 0;; ++spins) {
+      unsigned int v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (static_cast<int>(v - target) >= 0) break;
+      if (spins >= kSpinLimit) {
+        good = false;
+        raise_flag(status, PLE_ERR_TIMEOUT);
+        break;
       }
     }
+    __threadfence();
+    ok = good;
+  }
+  __syncthreads();
+  return ok;
+}
+
+struct SortArgs {
+  const int64_t* rows;
+  int64_t N;
+  int64_t num_rows;
+  uint32_t* keys[2];
+  uint32_t* vals[2];
+  uint32_t* hist[2];  // [blocks][256] per pass parity
+  uint32_t* off;    // [blocks][256]
+  uint32_t* total;  // [256]
+  unsigned int* bar;
+  unsigned int* status;
+  int passes;
+};
+
+__global__ void __launch_bounds__(kCoopThreads) sort_kernel(const SortArgs a) {
+  __shared__ uint32_t h[kRadix];
+  __shared__ uint32_t wh[kCoopWarps][kRadix];
+  __shared__ uint32_t base_s[kRadix];
+  __shared__ uint32_t warp_tot[kCoopWarps];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t G = gridDim.x, b = blockIdx.x, N = a.N;
+  const int64_t seg = ((N + G - 1) / G + 31) / 32 * 32;
+  const int64_t lo = min(N, b * seg), hi = min(N, lo + seg);
+  bool bad = false;
+
+  // H (first pass only; later passes get their histograms from the previous
+  // scatter): histogram of this block's positions, making the keys
+  if (tid < kRadix) h[tid] = 0;
+  __syncthreads();
+  for (int64_t i0 = lo; i0 < hi; i0 += kCoopTile) {
+    uint32_t key[kCoopItems];
+#pragma unroll
+    for (int r = 0; r < kCoopItems; ++r) {  // every load first
+      const int64_t i = i0 + r * kCoopThreads + tid;
+      key[r] = 0;
+      if (i < hi) {
+        const int64_t v = a.rows[i];
+        const bool ok = v >= 0 && v < a.num_rows;
+        bad |= !ok;
+        key[r] = ok ? static_cast<uint32_t>(v) : static_cast<uint32_t>(a.num_rows);
+        a.keys[0][i] = key[r];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kCoopItems; ++r)
+      hist_add(h, i0 + r * kCoopThreads + tid < hi, key[r] & (kRadix - 1));
+  }
+  if (bad) raise_flag(a.status, PLE_ERR_BAD_ROW);
+  __syncthreads();
+  if (tid < kRadix) a.hist[0][b * kRadix + tid] = h[tid];
+  if (!grid_barrier(a.bar, a.status)) return;
+
+  for (int p = 0; p < a.passes; ++p) {
+    const int shift = 8 * p;
+    const bool odd = p & 1, last = p + 1 == a.passes;
+    const uint32_t* kin = odd ? a.keys[1] : a.keys[0];
+    const uint32_t* vin = odd ? a.vals[1] : a.vals[0];
+    uint32_t* kout = odd ? a.keys[0] : a.keys[1];
+    uint32_t* vout = odd ? a.vals[0] : a.vals[1];
+    const uint32_t* hist = odd ? a.hist[1] : a.hist[0];
+    uint32_t* hist_next = odd ? a.hist[0] : a.hist[1];
+
+    // P: per digit, exclusive scan over the blocks (two blocks per thread);
+    // every block also clears its row of the next pass's histogram
+    for (int d = static_cast<int>(b); d < kRadix; d += static_cast<int>(G)) {
+      const int64_t b0 = 2 * tid, b1 = 2 * tid + 1;
+      const uint32_t v0 = b0 < G ? __ldcg(hist + b0 * kRadix + d) : 0;
+      const uint32_t v1 = b1 < G ? __ldcg(hist + b1 * kRadix + d) : 0;
+      uint32_t tot;
+      const uint32_t ex = block_exclusive_sum(v0 + v1, warp_tot, &tot);
+      if (b0 < G) a.off[b0 * kRadix + d] = ex;
+      if (b1 < G) a.off[b1 * kRadix + d] = ex + v0;
+      if (tid == 0) a.total[d] = tot;
+    }
+    if (!last && tid < kRadix) hist_next[b * kRadix + tid] = 0;
+    if (!grid_barrier(a.bar, a.status)) return;
+
+    // S: stable scatter of this block's positions, tile by tile
+    uint32_t key[kCoopItems], val[kCoopItems];
+    auto load_tile = [&](int64_t i0) {
+#pragma unroll
+      for (int r = 0; r < kCoopItems; ++r) {
+        const int64_t i = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane;
+        key[r] = i < hi ? kin[i] : 0;
+        val[r] = i < hi ? (p == 0 ? static_cast<uint32_t>(i) : vin[i]) : 0;
+      }
+    };
+    if (lo < hi) load_tile(lo);  // in flight during the digit-base scan
+    {
+      const uint32_t t = tid < kRadix ? __ldcg(a.total + tid) : 0;
+      const uint32_t mine = tid < kRadix ? __ldcg(a.off + b * kRadix + tid) : 0;
+      uint32_t all;
+      const uint32_t digit_base = block_exclusive_sum(t, warp_tot, &all);
+      if (tid < kRadix) base_s[tid] = digit_base + mine;
+    }
+    for (int64_t i0 = lo; i0 < hi; i0 += kCoopTile) {
+      for (int k = tid; k < kCoopWarps * kRadix; k += kCoopThreads) (&wh[0][0])[k] = 0;
+      __syncthreads();
+      uint8_t rank[kCoopItems];
+#pragma unroll
+      for (int r = 0; r < kCoopItems; ++r) {
+        const bool valid = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi;
+        const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
+        const unsigned peers = peers_of<8>(valid, digit);
+        const unsigned lower = __popc(peers & lanemask_lt());
+        rank[r] = valid ? static_cast<uint8_t>(wh[warp][digit] + lower) : 0;
+        __syncwarp();
+        if (valid && lower == 0) wh[warp][digit] += __popc(peers);
+        __syncwarp();
+      }
+      __syncthreads();
+      uint32_t tile_count = 0;
+      if (tid < kRadix) {
+#pragma unroll
+        for (int w = 0; w < kCoopWarps; ++w) {
+          const uint32_t c = wh[w][tid];
+          wh[w][tid] = tile_count;
+          tile_count += c;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < kCoopItems; ++r) {
+        const bool valid = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi;
+        const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
+        const uint32_t dst = valid ? base_s[digit] + wh[warp][digit] + rank[r] : 0;
+        const bool write = valid && dst < N;  // dst < N always holds when the counts are consistent
+        if (write) {
+          kout[dst] = key[r];
+          vout[dst] = val[r];
+        }
+        if (!last) {  // histogram of the next pass, by destination block
+          const uint32_t cell = write ? static_cast<uint32_t>(dst / seg) * kRadix + ((key[r] >> (shift + 8)) & (kRadix - 1))
+                                      : 0xffffffffu;
+          const unsigned peers = __match_any_sync(kFull, cell);
+          if (write && (peers & lanemask_lt()) == 0) atomicAdd(hist_next + cell, __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (tid < kRadix) base_s[tid] += tile_count;
+      if (i0 + kCoopTile < hi) load_tile(i0 + kCoopTile);
+    }
+    if (!last && !grid_barrier(a.bar, a.status)) return;
   }
 }
 
@@ -392,6 +415,11 @@ __device__ int64_t find_run_start(const uint32_t* __restrict__ K, int64_t p, uin
   return hi;
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gmem_src) : "memory");
+}
+
 // Level 1 works on windows of 32 sorted positions, one warp per window.
 // One round trip brings the window's keys and hit indices, the next 32 keys
 // (a chunk that starts in this window may end in the next) and the previous
@@ -495,114 +523,85 @@ __device__ __forceinline__ void unpack16(const uint4& y, float* v) {
   }
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gmem_src) : "memory");
+// Wide fold.  A grad row spans L lanes that each copy 16 bytes, so one copy
+// instruction fetches 32/L rows; all rows of the window's positions [a, b)
+// (at most 63) are staged in shared memory with asynchronous copies in one
+// round trip.  The L-lane groups of the warp then take the window's chunks
+// in turn (chunk k to group k mod 32/L) and fold them independently from
+// shared memory, each group in the fixed order, lane `sub` of a group owning
+// CPLN = 16/elem columns.  A finished chunk that is a whole run is added into
+// table_grad by its group; otherwise it goes to its chunk-sum slot.
+constexpr int kWideRows = 64;  // staged rows per warp (a window covers at most 63)
+
+template <int L>
+__host__ __device__ constexpr int wide_warps() {
+  return L >= 32 ? 1 : L >= 16 ? 2 : 4;  // about <= 48 KB of staging per block
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+template <int L>
+__host__ __device__ constexpr size_t wide_smem() {
+  return static_cast<size_t>(wide_warps<L>()) * (kWideRows * L * 16 + kWideRows * 4);
 }
 
-constexpr int kWideWarps = 4;  // warps per block of the wide fold
-constexpr int kWideLoads = 8;  // 16-byte async copies per lane per batch
-
-// Wide fold: a grad row spans L lanes that each copy 16 bytes, so one
-// instruction fetches 32/L rows.  A batch of rows is staged in shared memory
-// by asynchronous copies (no registers held while they are in flight).  A run
-// of a single hit is added into table_grad by the lane group that fetched it.
-// Hits of longer runs are folded in order: every L-lane group keeps the same
-// running chunk sum (lane `sub` of a group owns CPLN = 16/elem columns) and
-// adds row after row from the staging buffer; the groups write finished
-// chunks in turn.
 template <int L, bool BF16>
-__global__ void __launch_bounds__(kWideWarps * 32, 8)
+__global__ void __launch_bounds__(wide_warps<L>() * 32)
 fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
                  const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
                  int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
-  constexpr int RPI = 32 / L;                                            // rows per copy instruction
-  constexpr int CPLN = BF16 ? 8 : 4;                                     // fp32 columns per lane
-  constexpr int BATCH = kWideLoads * RPI < 64 ? kWideLoads * RPI : 64;   // hits per batch
-  constexpr int LOADS = BATCH / RPI;                                     // copies per lane per batch
-  __shared__ uint4 stage[kWideWarps][kWideLoads][32];
+  constexpr int RPI = 32 / L;         // rows per copy instruction = lane groups per warp
+  constexpr int CPLN = BF16 ? 8 : 4;  // fp32 columns per lane
+  extern __shared__ __align__(16) unsigned char wide_smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / L, sub = lane % L;
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWideWarps + warp;
+  uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw) + warp * (kWideRows * L + kWideRows / 4);
+  uint32_t* keys_s = reinterpret_cast<uint32_t*>(rows_s + kWideRows * L);
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * wide_warps<L>() + warp;
+  wait_for_prior_grid();
+  allow_next_grid();
   if (w * 32 >= N) return;
   Window W;
   if (!window_setup(K, I, N, w, W)) return;
   const size_t row_bytes = static_cast<size_t>(D) * (BF16 ? 2 : 4);
   const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
-  // positions holding a run of exactly one hit
-  const uint64_t next_is_head = (W.hm >> 1) | (W.p0 + 63 >= N ? (1ull << (N - 1 - W.p0)) : 0ull);
-  const uint64_t single = W.hm & next_is_head;
 
-  float acc[CPLN];
-#pragma unroll
-  for (int k = 0; k < CPLN; ++k) acc[k] = 0.f;
-  int c = W.a, turn = 0;
-  for (int e0 = W.a; e0 < W.b; e0 += BATCH) {
-#pragma unroll
-    for (int s = 0; s < LOADS; ++s) {
-      const int e = e0 + s * RPI + grp;
-      const int src = e & 31;
-      const uint32_t ia = __shfl_sync(kFull, W.iA, src), ib = __shfl_sync(kFull, W.iB, src);
-      if (e < W.b) cp_async16(&stage[warp][s][lane], gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
-    }
-    cp_async_wait_all();
-    __syncwarp();
-#pragma unroll
-    for (int s = 0; s < LOADS; ++s) {
-      const int e = e0 + s * RPI + grp;
-      const int src = e & 31;
-      const uint32_t ka = __shfl_sync(kFull, W.kA, src), kb = __shfl_sync(kFull, W.kB, src);
-      const uint32_t key = e < 32 ? ka : kb;
-      if (e < W.b && ((single >> e) & 1ull) && key != bad_key) {
-        float v[CPLN];
-        unpack16<BF16>(stage[warp][s][lane], v);
-        float* dst = table_grad + static_cast<int64_t>(key) * D + sub * CPLN;
-#pragma unroll
-        for (int k = 0; k < CPLN; k += 4) red_add4(dst + k, v[k], v[k + 1], v[k + 2], v[k + 3]);
-      }
-    }
-    const int nb = min(BATCH, W.b - e0);
-    uint64_t multi = (~single >> e0) & (nb >= 64 ? ~0ull : ((1ull << nb) - 1));
-    while (multi) {
-      const int t = __ffsll(static_cast<long long>(multi)) - 1;
-      multi &= multi - 1;
-      const int e = e0 + t;
+  keys_s[lane] = W.kA;
+  keys_s[32 + lane] = W.kB;
+  for (int e0 = W.a; e0 < W.b; e0 += RPI) {  // uniform trip count: the shuffles see every lane
+    const int e = e0 + grp;
+    const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
+    if (e < W.b) cp_async16(rows_s + e * L + sub, gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+
+  const uint64_t in_range = (W.b >= 64 ? ~0ull : ((1ull << W.b) - 1)) & ~((1ull << W.a) - 1);
+  uint64_t starts = W.cm & in_range;  // chunk starts folded by this warp
+  int k = 0;
+  while (starts) {
+    const int c = __ffsll(static_cast<long long>(starts)) - 1;
+    starts &= starts - 1;
+    if ((k++ % RPI) != grp) continue;  // another group's chunk
+    const int nxt = starts ? __ffsll(static_cast<long long>(starts)) - 1 : W.b;
+    float acc[CPLN];
+    unpack16<BF16>(rows_s[c * L + sub], acc);
+    for (int e = c + 1; e < nxt; ++e) {
       float v[CPLN];
-      unpack16<BF16>(stage[warp][t / RPI][sub + L * (t % RPI)], v);
-      if ((W.cm >> e) & 1ull) {
-        c = e;
+      unpack16<BF16>(rows_s[e * L + sub], v);
 #pragma unroll
-        for (int k = 0; k < CPLN; ++k) acc[k] = v[k];
-      } else {
-#pragma unroll
-        for (int k = 0; k < CPLN; ++k) acc[k] = acc[k] + v[k];
-      }
-      const int nxt = e + 1;
-      if (nxt == W.b || ((W.cm >> nxt) & 1ull)) {  // chunk [c, nxt) complete
-        const uint32_t key = W.key_at(c);
-        if (key != bad_key) {
-          const int writer = turn % RPI;
-          int64_t slot = 0;
-          const bool whole = chunk_is_whole_run(W, c, nxt, N, lane == 0, &slot, mc_len, mc_list, mc_count);
-          if (grp == writer) {
-            float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
-            if (whole) {
-#pragma unroll
-              for (int k = 0; k < CPLN; k += 4) red_add4(dst + k, acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
-            } else {
-#pragma unroll
-              for (int k = 0; k < CPLN; k += 4)
-                *reinterpret_cast<float4*>(dst + k) = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
-            }
-          }
-          ++turn;
-        }
-      }
+      for (int q = 0; q < CPLN; ++q) acc[q] = acc[q] + v[q];
     }
-    __syncwarp();  // the next batch reuses the staging buffer
+    const uint32_t key = keys_s[c];
+    if (key == bad_key) continue;
+    int64_t slot = 0;
+    const bool whole = chunk_is_whole_run(W, c, nxt, N, sub == 0, &slot, mc_len, mc_list, mc_count);
+    float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
+    if (whole) {
+#pragma unroll
+      for (int q = 0; q < CPLN; q += 4) red_add4(dst + q, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < CPLN; q += 4)
+        *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+    }
   }
 }
 
@@ -616,6 +615,8 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
   constexpr int kBatch = 4;
   const int lane = threadIdx.x & 31;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5;
+  wait_for_prior_grid();
+  allow_next_grid();
   if (w * 32 >= N) return;
   Window W;
   if (!window_setup(K, I, N, w, W)) return;
@@ -661,13 +662,17 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
   }
 }
 
-// Level 2: one warp per run longer than 32 hits.
+// Level 2: one warp per run longer than 32 hits folds the run's chunk sums in
+// order (loads issued kAhead at a time ahead of the adds); one final add into
+// table_grad.
 template <int CPL>
 __global__ void __launch_bounds__(kFoldThreads)
 fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, const float* __restrict__ csum,
                   const int* __restrict__ mc_len, const int* __restrict__ mc_list, const int* __restrict__ mc_count,
                   int D, float* __restrict__ table_grad) {
+  constexpr int kAhead = CPL == 1 ? 32 : CPL == 2 ? 24 : CPL == 4 ? 16 : 8;
   const int lane = threadIdx.x & 31;
+  wait_for_prior_grid();
   const int count = *mc_count;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kFoldThreads / 32);
   for (int64_t q = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5; q < count; q += nwarps) {
@@ -676,7 +681,6 @@ fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, c
     const int nc = static_cast<int>((len + kChunk - 1) / kChunk);
     const uint32_t key = K[c0];
     if (key >= bad_key) continue;
-    Cols<CPL> acc;
     auto load_slot = [&](int64_t slot, Cols<CPL>& y) {
       if constexpr (CPL == 0) {
 #pragma unroll
@@ -688,8 +692,8 @@ fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, c
         for (int k = 0; k < CPL; ++k) y.v[k] = p[k];
       }
     };
+    Cols<CPL> acc;
     load_slot(2 * (c0 >> 5) + 1, acc);
-    constexpr int kAhead = 8;  // chunk sums loaded ahead of the in-order adds
     for (int m0 = 1; m0 < nc; m0 += kAhead) {
       Cols<CPL> y[kAhead];
 #pragma unroll
@@ -730,9 +734,8 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
 // host side
 // ---------------------------------------------------------------------------
 struct Layout {
-  size_t keys[2], vals[2], hist, gtot, csum, mc_len, mc_list, zeroed, total;
-  size_t zeroed_bytes;  // tickets of every pass + the heavy-run counter, cleared per call
-  int num_tiles, num_groups, max_passes;
+  size_t keys[2], vals[2], hist[2], off, total, csum, mc_len, mc_list, zeroed, total_bytes;
+  size_t zeroed_bytes;  // the sort's barrier counter and the heavy-run counter, cleared per call
   int64_t nwin;
 };
 
@@ -740,9 +743,6 @@ size_t align_up(size_t x) { return (x + 255) & ~size_t{255}; }
 
 Layout layout_for(int64_t N, int D) {
   Layout L{};
-  L.num_tiles = static_cast<int>((N + kSortTile - 1) / kSortTile);
-  L.num_groups = (L.num_tiles + kTilesPerGroup - 1) / kTilesPerGroup;
-  L.max_passes = 4;
   L.nwin = (N + 31) / 32;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -752,15 +752,35 @@ Layout layout_for(int64_t N, int D) {
   };
   for (int b = 0; b < 2; ++b) L.keys[b] = take(sizeof(uint32_t) * N);
   for (int b = 0; b < 2; ++b) L.vals[b] = take(sizeof(uint32_t) * N);
-  L.hist = take(sizeof(uint32_t) * kRadix * static_cast<size_t>(L.num_tiles));
-  L.gtot = take(sizeof(uint32_t) * kRadix * static_cast<size_t>(L.num_groups));
+  L.hist[0] = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
+  L.hist[1] = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
+  L.off = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
+  L.total = take(sizeof(uint32_t) * kRadix);
   L.csum = take(sizeof(float) * 2 * static_cast<size_t>(L.nwin) * D);
   L.mc_len = take(sizeof(int) * L.nwin);
   L.mc_list = take(sizeof(int) * L.nwin);
-  L.zeroed_bytes = sizeof(unsigned int) * (static_cast<size_t>(L.max_passes) * (L.num_groups + 1) + 1);
+  L.zeroed_bytes = 2 * sizeof(unsigned int);
   L.zeroed = take(L.zeroed_bytes);
-  L.total = off;
+  L.total_bytes = off;
   return L;
+}
+
+// Blocks of the cooperative sort: all resident at once, at most one tile each
+// when the input is small.
+int sort_blocks(int64_t N, cudaError_t* err) {
+  static std::atomic<int> per_sm_cache[64];
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return 0;
+  int per_sm = (dev >= 0 && dev < 64) ? per_sm_cache[dev].load(std::memory_order_relaxed) : 0;
+  if (per_sm <= 0) {
+    *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sort_kernel, kCoopThreads, 0);
+    if (*err != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) per_sm_cache[dev].store(per_sm, std::memory_order_relaxed);
+  }
+  const int64_t resident = static_cast<int64_t>(per_sm) * sm_count();
+  const int64_t tiles = (N + kCoopTile - 1) / kCoopTile;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({resident, tiles, int64_t{kCoopMaxBlocks}})));
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -792,7 +812,7 @@ extern "C" {
 
 size_t ple_grad_scatter_workspace_bytes(const ple_plan_t* plan, int64_t N) {
   if (plan == nullptr || N <= 0) return 0;
-  return layout_for(N, plan->head_dim).total;
+  return layout_for(N, plan->head_dim).total_bytes;
 }
 
 ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* grad,
@@ -803,88 +823,84 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   if (plan->num_rows >= static_cast<int64_t>(kNoKey) || N >= (int64_t{1} << 31)) return PLE_ERR_UNSUPPORTED;
   const int D = plan->head_dim;
   const Layout L = layout_for(N, D);
-  if (workspace == nullptr || ws_bytes < L.total) return PLE_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < L.total_bytes) return PLE_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
   unsigned int* status = status_word(&e);
   if (status == nullptr) return cuda_fail(e);
   auto* ws = static_cast<unsigned char*>(workspace);
-  uint32_t* keys[2] = {reinterpret_cast<uint32_t*>(ws + L.keys[0]), reinterpret_cast<uint32_t*>(ws + L.keys[1])};
-  uint32_t* vals[2] = {reinterpret_cast<uint32_t*>(ws + L.vals[0]), reinterpret_cast<uint32_t*>(ws + L.vals[1])};
-  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-  uint32_t* gtot = reinterpret_cast<uint32_t*>(ws + L.gtot);
+  const auto s = static_cast<cudaStream_t>(stream);
+  SortArgs sa{};
+  sa.rows = rows;
+  sa.N = N;
+  sa.num_rows = plan->num_rows;
+  for (int b = 0; b < 2; ++b) {
+    sa.keys[b] = reinterpret_cast<uint32_t*>(ws + L.keys[b]);
+    sa.vals[b] = reinterpret_cast<uint32_t*>(ws + L.vals[b]);
+  }
+  sa.hist[0] = reinterpret_cast<uint32_t*>(ws + L.hist[0]);
+  sa.hist[1] = reinterpret_cast<uint32_t*>(ws + L.hist[1]);
+  sa.off = reinterpret_cast<uint32_t*>(ws + L.off);
+  sa.total = reinterpret_cast<uint32_t*>(ws + L.total);
+  sa.bar = reinterpret_cast<unsigned int*>(ws + L.zeroed);
+  sa.status = status;
   float* csum = reinterpret_cast<float*>(ws + L.csum);
   int* mc_len = reinterpret_cast<int*>(ws + L.mc_len);
   int* mc_list = reinterpret_cast<int*>(ws + L.mc_list);
-  unsigned int* tickets = reinterpret_cast<unsigned int*>(ws + L.zeroed);
-  int* mc_count = reinterpret_cast<int*>(tickets + static_cast<size_t>(L.max_passes) * (L.num_groups + 1));
-  const auto s = static_cast<cudaStream_t>(stream);
+  int* mc_count = reinterpret_cast<int*>(sa.bar + 1);
 
   // key bits: keys lie in [0, num_rows] (num_rows marks a bad row)
   int bits = 0;
   while (bits < 32 && (static_cast<uint64_t>(plan->num_rows) >> bits) != 0) ++bits;
-  const int passes = (bits + 7) / 8;
+  sa.passes = std::max(1, (bits + 7) / 8);
 
-  e = cudaMemsetAsync(tickets, 0, L.zeroed_bytes, s);
+  e = cudaMemsetAsync(sa.bar, 0, L.zeroed_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  keys_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(rows, N, plan->num_rows, keys[0], hist, gtot, tickets,
-                                                   L.num_tiles, status);
-  int cur = 0;
-  for (int p = 0; p < passes; ++p) {
-    if (p > 0)
-      hist_kernel<<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], N, 8 * p, hist, gtot,
-                                                       tickets + static_cast<size_t>(p) * (L.num_groups + 1),
-                                                       L.num_tiles);
-    if (p == 0)
-      scatter_kernel<true><<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], nullptr, keys[1 - cur], vals[1 - cur],
-                                                                hist, gtot, N, 0, L.num_tiles);
-    else
-      scatter_kernel<false><<<L.num_tiles, kSortThreads, 0, s>>>(keys[cur], vals[cur], keys[1 - cur],
-                                                                 vals[1 - cur], hist, gtot, N, 8 * p, L.num_tiles);
-    cur = 1 - cur;
-  }
-  const uint32_t* Ks = keys[cur];
-  const uint32_t* Is = vals[cur];
+  const int blocks = sort_blocks(N, &e);
+  if (blocks <= 0) return cuda_fail(e);
+  void* kargs[] = {&sa};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(sort_kernel), dim3(blocks), dim3(kCoopThreads),
+                                  kargs, 0, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const uint32_t* Ks = sa.keys[sa.passes & 1];
+  const uint32_t* Is = sa.vals[sa.passes & 1];
   const uint32_t bad_key = static_cast<uint32_t>(plan->num_rows);
-  const unsigned fold_blocks = static_cast<unsigned>((L.nwin * 32 + kFoldThreads - 1) / kFoldThreads);
-  const unsigned heavy_blocks = static_cast<unsigned>(sm_count() * 4);
+  const dim3 fold_grid(static_cast<unsigned>((L.nwin * 32 + kFoldThreads - 1) / kFoldThreads));
   const bool bf = gdt == PLE_BF16;
   const int lanes_per_row = static_cast<int>(static_cast<int64_t>(D) * (bf ? 2 : 4) / 16);
-  const unsigned wide_blocks = static_cast<unsigned>((L.nwin + kWideWarps - 1) / kWideWarps);
-#define PLE_FOLD_WIDE(LW)                                                                                   \
-  case LW:                                                                                                  \
-    if (bf)                                                                                                 \
-      fold_wide_kernel<LW, true><<<wide_blocks, kWideWarps * 32, 0, s>>>(Ks, Is, N, bad_key, grad, D,       \
-                                                                         table_grad, csum, mc_len, mc_list, \
-                                                                         mc_count);                         \
-    else                                                                                                    \
-      fold_wide_kernel<LW, false><<<wide_blocks, kWideWarps * 32, 0, s>>>(Ks, Is, N, bad_key, grad, D,      \
-                                                                          table_grad, csum, mc_len, mc_list, \
-                                                                          mc_count);                        \
+  auto fold = [&](auto kernel, dim3 grid, int threads, size_t smem) {
+    return launch_after(kernel, grid, dim3(threads), smem, s, Ks, Is, N, bad_key, grad, D, table_grad, csum,
+                        mc_len, mc_list, mc_count);
+  };
+#define PLE_WIDE(LW, BF)                                                                                  \
+  case 2 * LW + BF:                                                                                       \
+    e = fold(fold_wide_kernel<LW, BF>,                                                                    \
+             dim3(static_cast<unsigned>((L.nwin + wide_warps<LW>() - 1) / wide_warps<LW>())),            \
+             wide_warps<LW>() * 32, wide_smem<LW>());                                                     \
     break;
-  switch (lanes_per_row) {
-    PLE_FOLD_WIDE(1)
-    PLE_FOLD_WIDE(2)
-    PLE_FOLD_WIDE(4)
-    PLE_FOLD_WIDE(8)
-    PLE_FOLD_WIDE(16)
-    PLE_FOLD_WIDE(32)
+  switch (lanes_per_row * 2 + (bf ? 1 : 0)) {
+    PLE_WIDE(1, 0) PLE_WIDE(1, 1) PLE_WIDE(2, 0) PLE_WIDE(2, 1) PLE_WIDE(4, 0) PLE_WIDE(4, 1)
+    PLE_WIDE(8, 0) PLE_WIDE(8, 1) PLE_WIDE(16, 0) PLE_WIDE(16, 1) PLE_WIDE(32, 0) PLE_WIDE(32, 1)
     default:
-      if (bf)
-        fold_generic_kernel<true><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad,
-                                                                       csum, mc_len, mc_list, mc_count);
-      else
-        fold_generic_kernel<false><<<fold_blocks, kFoldThreads, 0, s>>>(Ks, Is, N, bad_key, grad, D, table_grad,
-                                                                        csum, mc_len, mc_list, mc_count);
+      e = bf ? fold(fold_generic_kernel<true>, fold_grid, kFoldThreads, 0)
+             : fold(fold_generic_kernel<false>, fold_grid, kFoldThreads, 0);
   }
-#undef PLE_FOLD_WIDE
+#undef PLE_WIDE
+  if (e != cudaSuccess) return cuda_fail(e);
+  const dim3 heavy_grid(static_cast<unsigned>(sm_count() * 4));
+  auto heavy = [&](auto kernel) {
+    return launch_after(kernel, heavy_grid, dim3(kFoldThreads), 0, s, Ks, N, bad_key,
+                        static_cast<const float*>(csum), static_cast<const int*>(mc_len),
+                        static_cast<const int*>(mc_list), static_cast<const int*>(mc_count), D, table_grad);
+  };
   switch (cols_per_lane(D)) {
-    case 1: fold_heavy_kernel<1><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
-    case 2: fold_heavy_kernel<2><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
-    case 4: fold_heavy_kernel<4><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
-    case 8: fold_heavy_kernel<8><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
-    default: fold_heavy_kernel<0><<<heavy_blocks, kFoldThreads, 0, s>>>(Ks, N, bad_key, csum, mc_len, mc_list, mc_count, D, table_grad); break;
+    case 1: e = heavy(fold_heavy_kernel<1>); break;
+    case 2: e = heavy(fold_heavy_kernel<2>); break;
+    case 4: e = heavy(fold_heavy_kernel<4>); break;
+    case 8: e = heavy(fold_heavy_kernel<8>); break;
+    default: e = heavy(fold_heavy_kernel<0>); break;
   }
+  if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
 

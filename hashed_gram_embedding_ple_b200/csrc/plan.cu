@@ -154,6 +154,7 @@ const char* ple_strerror(ple_status_t s) {
     case PLE_ERR_CUDA: return "CUDA runtime error";
     case PLE_ERR_BAD_ROW: return "row id outside the table (output zeroed or hit dropped)";
     case PLE_ERR_BAD_SEQLENS: return "malformed cu_seqlens";
+    case PLE_ERR_TIMEOUT: return "a bounded wait between blocks ran out (results unspecified)";
   }
   return "unknown status";
 }

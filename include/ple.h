@@ -57,7 +57,8 @@ typedef enum {
   PLE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
   PLE_ERR_CUDA = 5,          /* CUDA runtime error; see ple_last_cuda_error */
   PLE_ERR_BAD_ROW = 6,       /* async: a row id outside [0, num_rows) */
-  PLE_ERR_BAD_SEQLENS = 7    /* async: cu_seqlens not 0..num_tokens, or decreasing */
+  PLE_ERR_BAD_SEQLENS = 7,   /* async: cu_seqlens not 0..num_tokens, or decreasing */
+  PLE_ERR_TIMEOUT = 8        /* async: a bounded wait between the blocks of a kernel ran out */
 } ple_status_t;
 
 typedef enum { PLE_F32 = 0, PLE_BF16 = 1 } ple_dtype_t;
