@@ -60,7 +60,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // The barrier's wait is bounded: past the limit the block raises
 // PLE_ERR_TIMEOUT and leaves (the result is then unspecified, nothing hangs).
 // ---------------------------------------------------------------------------
-constexpr int kCoopThreads = 512;
+constexpr int kCoopThreads = 256;
 constexpr int kCoopWarps = kCoopThreads / 32;
 constexpr int kCoopItems = 4;
 constexpr int kCoopTile = kCoopThreads * kCoopItems;  // keys per tile of the scatter phase
@@ -153,10 +153,13 @@ struct SortArgs {
   int passes;
 };
 
-__global__ void __launch_bounds__(kCoopThreads) sort_kernel(const SortArgs a) {
+__global__ void __launch_bounds__(kCoopThreads, 4) sort_kernel(const SortArgs a) {
   __shared__ uint32_t h[kRadix];
   __shared__ uint32_t wh[kCoopWarps][kRadix];
   __shared__ uint32_t base_s[kRadix];
+  __shared__ uint32_t start_s[kRadix];
+  __shared__ uint32_t stage_k[kCoopTile];
+  __shared__ uint32_t stage_v[kCoopTile];
   __shared__ uint32_t warp_tot[kCoopWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t G = gridDim.x, b = blockIdx.x, N = a.N;
@@ -259,22 +262,31 @@ __global__ void __launch_bounds__(kCoopThreads) sort_kernel(const SortArgs a) {
           tile_count += c;
         }
       }
+      // tile-local start of every digit, then stage the tile in digit order
+      uint32_t tile_n;
+      const uint32_t local_start = block_exclusive_sum(tid < kRadix ? tile_count : 0u, warp_tot, &tile_n);
+      if (tid < kRadix) start_s[tid] = local_start;
       __syncthreads();
 #pragma unroll
       for (int r = 0; r < kCoopItems; ++r) {
-        const bool valid = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi;
-        const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-        const uint32_t dst = valid ? base_s[digit] + wh[warp][digit] + rank[r] : 0;
-        const bool write = valid && dst < N;  // dst < N always holds when the counts are consistent
-        if (write) {
-          kout[dst] = key[r];
-          vout[dst] = val[r];
+        if (i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi) {
+          const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
+          const uint32_t pos = start_s[digit] + wh[warp][digit] + rank[r];
+          stage_k[pos] = key[r];
+          stage_v[pos] = val[r];
         }
-        if (!last) {  // histogram of the next pass, by destination block
-          const uint32_t cell = write ? static_cast<uint32_t>(dst / seg) * kRadix + ((key[r] >> (shift + 8)) & (kRadix - 1))
-                                      : 0xffffffffu;
-          const unsigned peers = __match_any_sync(kFull, cell);
-          if (write && (peers & lanemask_lt()) == 0) atomicAdd(hist_next + cell, __popc(peers));
+      }
+      __syncthreads();
+      // coalesced writes: consecutive threads, consecutive destinations within a digit
+      for (uint32_t j = tid; j < tile_n; j += kCoopThreads) {
+        const uint32_t k2 = stage_k[j];
+        const uint32_t digit = (k2 >> shift) & (kRadix - 1);
+        const uint32_t dst = base_s[digit] + (j - start_s[digit]);
+        if (dst < N) {  // always true when the counts are consistent
+          kout[dst] = k2;
+          vout[dst] = stage_v[j];
+          if (!last)  // histogram of the next pass, by destination block
+            atomicAdd(hist_next + static_cast<uint32_t>(dst / seg) * kRadix + ((k2 >> (shift + 8)) & (kRadix - 1)), 1u);
         }
       }
       __syncthreads();
