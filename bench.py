@@ -136,6 +136,22 @@ def traffic_from_profiles(key: str, source_files):
     return None
 
 
+def reduce_max(values, dist, device):
+    """Element-wise max over ranks (replica timings are taken as the slowest
+    rank's); a no-op without a process group."""
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own batch."""
+    return base + rank
+
+
 def cpu_oracle_step(w, table_host, grad_host, threads, tokens_limit=None):
     """The oracle, as it stands, on the first `tokens_limit` tokens (whole
     sequences cut at that point): rows, gather, gradient sums."""
@@ -240,7 +256,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w = workload(args.workload, args.seed + rank)  # each replica its own batch
+    w = workload(args.workload, replica_seed(args.seed, rank))
     plan = ple.Plan.from_workload(w)
     T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
     tdt = torch.bfloat16 if w.table_dtype == 1 else torch.float32
@@ -313,11 +329,8 @@ def main():
     fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
     bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
     step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
-    local = torch.tensor([statistics.mean(step_ms), statistics.mean(fwd_ms), statistics.mean(bwd_ms)],
-                         dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(local, op=dist.ReduceOp.MAX)
-    ms_step, ms_fwd, ms_bwd = [float(x) for x in local.tolist()]
+    ms_step, ms_fwd, ms_bwd = reduce_max([statistics.mean(step_ms), statistics.mean(fwd_ms),
+                                          statistics.mean(bwd_ms)], dist, dev)
 
     peak, peak_kind = measured_peaks()
     e_t = 2 if w.table_dtype == 1 else 4
@@ -374,12 +387,10 @@ def main():
             torch.cuda.synchronize()
             if k >= 2:
                 times.append(e0.elapsed_time(e1))
-        t_e2e = torch.tensor([statistics.mean(times)], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+        (t_e2e_ms,) = reduce_max([statistics.mean(times)], dist, dev)
         h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
-        e2e = {"value": world * T / (float(t_e2e.item()) * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": N * D * e_t, "ms_per_step": float(t_e2e.item()),
+        e2e = {"value": world * T / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": N * D * e_t, "ms_per_step": t_e2e_ms,
                "what": "pinned H2D tokens+cu_seqlens+grad_out, ple_lookup, ple_grad_scatter, D2H of the lookup output"}
 
     cpu = None
