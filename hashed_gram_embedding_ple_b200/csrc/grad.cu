@@ -536,22 +536,24 @@ __device__ __forceinline__ void unpack16(const uint4& y, float* v) {
 }
 
 // Wide fold.  A grad row spans L lanes that each copy 16 bytes, so one copy
-// instruction fetches 32/L rows; all rows of the window's positions [a, b)
-// (at most 63) are staged in shared memory with asynchronous copies in one
-// round trip.  The L-lane groups of the warp then take the window's chunks
-// in turn (chunk k to group k mod 32/L) and fold them independently from
-// shared memory, each group in the fixed order, lane `sub` of a group owning
-// CPLN = 16/elem columns.  A finished chunk that is a whole run is added into
+// instruction fetches 32/L rows.  The chunks that start in the window are
+// taken in rounds of whole chunks covering at most kWideRows positions (a
+// chunk has at most 32 hits, so it never straddles two rounds); the rows of
+// a round are staged in shared memory with asynchronous copies in one round
+// trip.  The L-lane groups of the warp then take the round's chunks in turn
+// (chunk k to group k mod 32/L) and fold them independently from shared
+// memory, each in the fixed order, lane `sub` of a group owning CPLN =
+// 16/elem columns.  A finished chunk that is a whole run is added into
 // table_grad by its group; otherwise it goes to its chunk-sum slot.
-constexpr int kWideRows = 64;  // staged rows per warp (a window covers at most 63)
+constexpr int kWideRows = 32;  // staged rows per warp and round
 
 template <int L>
 __host__ __device__ constexpr int wide_warps() {
-  return L >= 32 ? 1 : L >= 16 ? 2 : 4;  // about <= 48 KB of staging per block
+  return L >= 32 ? 2 : L >= 16 ? 4 : 8;  // about 33 KB of staging per block
 }
 template <int L>
 __host__ __device__ constexpr size_t wide_smem() {
-  return static_cast<size_t>(wide_warps<L>()) * (kWideRows * L * 16 + kWideRows * 4);
+  return static_cast<size_t>(wide_warps<L>()) * (kWideRows * L * 16 + 64 * 4);
 }
 
 template <int L, bool BF16>
@@ -564,8 +566,8 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   extern __shared__ __align__(16) unsigned char wide_smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / L, sub = lane % L;
-  uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw) + warp * (kWideRows * L + kWideRows / 4);
-  uint32_t* keys_s = reinterpret_cast<uint32_t*>(rows_s + kWideRows * L);
+  uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw) + warp * (kWideRows * L + 16);
+  uint32_t* keys_s = reinterpret_cast<uint32_t*>(rows_s + kWideRows * L);  // 64 keys
   const int64_t w = static_cast<int64_t>(blockIdx.x) * wide_warps<L>() + warp;
   wait_for_prior_grid();
   allow_next_grid();
@@ -574,46 +576,58 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   if (!window_setup(K, I, N, w, W)) return;
   const size_t row_bytes = static_cast<size_t>(D) * (BF16 ? 2 : 4);
   const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
-
   keys_s[lane] = W.kA;
   keys_s[32 + lane] = W.kB;
-  for (int e0 = W.a; e0 < W.b; e0 += RPI) {  // uniform trip count: the shuffles see every lane
-    const int e = e0 + grp;
-    const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
-    if (e < W.b) cp_async16(rows_s + e * L + sub, gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
-  }
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-  __syncwarp();
 
   const uint64_t in_range = (W.b >= 64 ? ~0ull : ((1ull << W.b) - 1)) & ~((1ull << W.a) - 1);
-  uint64_t starts = W.cm & in_range;  // chunk starts folded by this warp
+  uint64_t rem = W.cm & in_range;  // chunk starts still to fold
   int k = 0;
-  while (starts) {
-    const int c = __ffsll(static_cast<long long>(starts)) - 1;
-    starts &= starts - 1;
-    if ((k++ % RPI) != grp) continue;  // another group's chunk
-    const int nxt = starts ? __ffsll(static_cast<long long>(starts)) - 1 : W.b;
-    float acc[CPLN];
-    unpack16<BF16>(rows_s[c * L + sub], acc);
-    for (int e = c + 1; e < nxt; ++e) {
-      float v[CPLN];
-      unpack16<BF16>(rows_s[e * L + sub], v);
-#pragma unroll
-      for (int q = 0; q < CPLN; ++q) acc[q] = acc[q] + v[q];
+  while (rem) {
+    // the round: whole chunks from the first remaining start, at most kWideRows positions
+    const int r0 = __ffsll(static_cast<long long>(rem)) - 1;
+    int r1 = W.b;
+    if (W.b - r0 > kWideRows) {
+      const uint64_t later = rem & ~(1ull << r0) & ((2ull << (r0 + kWideRows)) - 1);
+      r1 = 63 - __clzll(later);  // a later chunk start within reach exists: chunks are <= 32 long
     }
-    const uint32_t key = keys_s[c];
-    if (key == bad_key) continue;
-    int64_t slot = 0;
-    const bool whole = chunk_is_whole_run(W, c, nxt, N, sub == 0, &slot, mc_len, mc_list, mc_count);
-    float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
-    if (whole) {
-#pragma unroll
-      for (int q = 0; q < CPLN; q += 4) red_add4(dst + q, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
-    } else {
-#pragma unroll
-      for (int q = 0; q < CPLN; q += 4)
-        *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+    for (int i0 = 0; i0 < r1 - r0; i0 += RPI) {  // uniform trip count: the shuffles see every lane
+      const int e = r0 + i0 + grp;
+      const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
+      if (e < r1)
+        cp_async16(rows_s + (e - r0) * L + sub, gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    uint64_t starts = rem & ((r1 >= 64 ? ~0ull : ((1ull << r1) - 1)));
+    rem &= ~starts;
+    while (starts) {
+      const int c = __ffsll(static_cast<long long>(starts)) - 1;
+      starts &= starts - 1;
+      if ((k++ % RPI) != grp) continue;  // another group's chunk
+      const int nxt = starts ? __ffsll(static_cast<long long>(starts)) - 1 : r1;
+      float acc[CPLN];
+      unpack16<BF16>(rows_s[(c - r0) * L + sub], acc);
+      for (int e = c + 1; e < nxt; ++e) {
+        float v[CPLN];
+        unpack16<BF16>(rows_s[(e - r0) * L + sub], v);
+#pragma unroll
+        for (int q = 0; q < CPLN; ++q) acc[q] = acc[q] + v[q];
+      }
+      const uint32_t key = keys_s[c];
+      if (key == bad_key) continue;
+      int64_t slot = 0;
+      const bool whole = chunk_is_whole_run(W, c, nxt, N, sub == 0, &slot, mc_len, mc_list, mc_count);
+      float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
+      if (whole) {
+#pragma unroll
+        for (int q = 0; q < CPLN; q += 4) red_add4(dst + q, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < CPLN; q += 4)
+          *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+      }
+    }
+    __syncwarp();  // the next round reuses the staging buffer
   }
 }
 
