@@ -20,7 +20,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -358,8 +357,7 @@ def main():
         if ms_bwd > ms_fwd:
             roofline = bwd_roof
 
-    passes = math.ceil(max(1, int(w.num_rows).bit_length()) / 8)
-    launches_per_step = 1 + ((2 * passes + 2) if do_bwd else 0)  # lookup; keys, passes x scatter, passes-1 x hist, two folds
+    launches_per_step = 1 + (2 if do_bwd else 0)  # lookup_kernel; sort_kernel (all passes) and the fold kernel
     value = world * T / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers

@@ -9,19 +9,15 @@
 //   (fp32); the chunk sums summed left to right from the first; the row sum
 //   added once into table_grad[r].
 //
-// Pipeline (all in the caller's workspace, no allocation, no inter-block
-// waiting):
-//   1. keys_kernel: 32-bit keys from the int64 rows (bad rows -> key R),
-//      per-tile histogram of the first digit;
-//   2. LSD radix sort, 8-bit digits, stable (reduce-then-scan per pass:
-//      histogram, one-block exclusive scan, rank-and-scatter), values = i;
-//   3. fold_kernel: one warp per 32 sorted positions ("window"); finds the
-//      chunk starts in its window (a chunk start is a position whose offset
-//      from its run's first position is a multiple of 32), folds each chunk
-//      it starts, and either adds a whole single-chunk run into table_grad
-//      or stores the chunk sum in a slot of the workspace;
-//   4. fold_heavy_kernel: one warp per run longer than 32 folds its chunk
-//      sums in order and adds the result into table_grad.
+// Pipeline (all in the caller's workspace, no allocation):
+//   1. sort_kernel (cooperative): 32-bit keys from the int64 rows (bad rows
+//      -> key R), LSD radix sort with 8-bit digits, stable, values = hit index;
+//   2. fold kernel: one warp per window of 32 sorted positions; it folds the
+//      chunks that start in its window (a chunk start is a position whose
+//      offset from its run's first position is a multiple of 32), adds a
+//      whole single-chunk run into table_grad, or stores the chunk sum of a
+//      longer run in a slot; the writer that completes a long run (per-run
+//      counter) folds that run's chunk sums in order and adds the result.
 // The final add is a vector fp32 reduction (red.global.add) issued by the one
 // warp that owns the row, so it is the single add table_grad + S_r.
 #include <algorithm>
@@ -150,6 +146,8 @@ struct SortArgs {
   uint32_t* total;  // [256]
   unsigned int* bar;
   unsigned int* status;
+  unsigned int* run_done;  // [nwin] cleared here for the fold
+  int64_t nwin;
   int passes;
 };
 
@@ -166,6 +164,7 @@ __global__ void __launch_bounds__(kCoopThreads, 4) sort_kernel(const SortArgs a)
   const int64_t seg = ((N + G - 1) / G + 31) / 32 * 32;
   const int64_t lo = min(N, b * seg), hi = min(N, lo + seg);
   bool bad = false;
+  for (int64_t i = b * kCoopThreads + tid; i < a.nwin; i += G * kCoopThreads) a.run_done[i] = 0;
 
   // H (first pass only; later passes get their histograms from the previous
   // scatter): histogram of this block's positions, making the keys
@@ -498,26 +497,61 @@ __device__ __forceinline__ bool window_setup(const uint32_t* __restrict__ K, con
   return true;
 }
 
-// Bookkeeping of a finished chunk [c, nxt) (relative positions) whose sum the
-// calling lanes hold: returns true if the chunk is a whole run (the caller
-// adds it into table_grad), false if its sum goes to a chunk-sum slot
-// (returned in *slot); lane `leader` records heavy-run metadata.
-__device__ __forceinline__ bool chunk_is_whole_run(const Window& W, int c, int nxt, int64_t N, bool leader,
-                                                   int64_t* slot, int* __restrict__ mc_len,
-                                                   int* __restrict__ mc_list, int* __restrict__ mc_count) {
+// Runs longer than 32 hits: each chunk sum goes to a slot; the run is
+// identified by its first position s (no two such runs start in one 32-position
+// window).  Every chunk writer adds 1 to done[s/32], except the writer of the
+// run's last chunk, which knows the run's length and adds kDoneTarget - nc + 1
+// instead; so the counter reaches kDoneTarget exactly once, when every chunk
+// sum is stored, and the writer that brings it there folds the chunk sums in
+// order (second level) and makes the run's single final add.  Nobody waits.
+constexpr unsigned kDoneTarget = 1u << 30;
+
+struct RunBook {
+  int* len;        // [windows] run length, written by the last chunk's writer
+  unsigned* done;  // [windows] completion counters, cleared before the fold
+};
+
+__device__ __forceinline__ int64_t chunk_slot(int64_t s, int m) {
+  return m == 0 ? 2 * (s >> 5) + 1 : 2 * ((s + static_cast<int64_t>(m) * kChunk) >> 5);
+}
+
+// Where the sum of chunk [c, nxt) goes: a whole run -> returns true; else the
+// chunk-sum slot in *slot.
+__device__ __forceinline__ bool chunk_is_whole_run(const Window& W, int c, int nxt, int64_t N, int64_t* slot) {
   const bool is_head = (W.hm >> c) & 1ull;
   const bool run_ends = (W.p0 + nxt >= N) || ((W.hm >> nxt) & 1ull);
   if (is_head && run_ends) return true;
   const int64_t pos = W.p0 + c;
   *slot = 2 * (pos >> 5) + (is_head ? 1 : 0);
-  if (leader) {
-    if (is_head) mc_list[atomicAdd(mc_count, 1)] = static_cast<int>(pos);
-    if (run_ends) {
-      const int64_t s = W.run_start(c);
-      mc_len[s >> 5] = static_cast<int>(W.p0 + nxt - s);
-    }
-  }
   return false;
+}
+
+// Called by the lanes `gmask` (leader lane `leader`) after they stored the sum
+// of chunk [c, nxt) of a run longer than 32 in its slot.  Returns, to all of
+// them, the run's chunk count if this chunk completed the run, else 0.
+__device__ __forceinline__ int chunk_stored(const Window& W, int c, int nxt, int64_t N, unsigned gmask, int leader,
+                                            const RunBook& rb, int64_t* run_start) {
+  const int lane = threadIdx.x & 31;
+  const bool run_ends = (W.p0 + nxt >= N) || ((W.hm >> nxt) & 1ull);
+  const int64_t s = W.run_start(c);
+  *run_start = s;
+  __threadfence();  // this lane's part of the chunk sum, before the count
+  __syncwarp(gmask);
+  int nc = 0;
+  if (lane == leader) {
+    unsigned inc = 1;
+    if (run_ends) {
+      const int len = static_cast<int>(W.p0 + nxt - s);
+      rb.len[s >> 5] = len;
+      __threadfence();
+      inc = kDoneTarget - static_cast<unsigned>((len + kChunk - 1) / kChunk) + 1;
+    }
+    const unsigned old = atomicAdd(rb.done + (s >> 5), inc);
+    if (old + inc == kDoneTarget) nc = (__ldcg(rb.len + (s >> 5)) + kChunk - 1) / kChunk;
+  }
+  nc = __shfl_sync(gmask, nc, leader);
+  if (nc) __threadfence();  // the other writers' chunk sums, before reading them
+  return nc;
 }
 
 __device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
@@ -532,6 +566,46 @@ __device__ __forceinline__ void unpack16(const uint4& y, float* v) {
   } else {
     v[0] = __uint_as_float(y.x); v[1] = __uint_as_float(y.y);
     v[2] = __uint_as_float(y.z); v[3] = __uint_as_float(y.w);
+  }
+}
+
+// Second level of a long run, by a whole warp after its window is folded:
+// the run's chunk sums go through the warp's staging buffer (`stage_vecs`
+// 16-byte vectors) by asynchronous copies, a buffer-full per round trip, and
+// lane l adds column vectors l, l+32 of them in order; one final reduction.
+__device__ void finish_run_staged(const float* csum, int64_t s, int nc, int D, uint32_t key, float* table_grad,
+                                  uint4* stage, int stage_vecs) {
+  const int lane = threadIdx.x & 31;
+  const int vps = D / 4;                 // 16-byte vectors per chunk sum (D <= 256: <= 64)
+  const int cap = stage_vecs / vps;      // chunk sums per round (>= 16 for the wide fold's buffers)
+  float acc[2][4];
+  for (int m0 = 0; m0 < nc; m0 += cap) {
+    const int np = min(cap, nc - m0);
+    for (int v = lane; v < np * vps; v += 32) {
+      const int m = m0 + v / vps, col = v % vps;
+      cp_async16(stage + v, csum + chunk_slot(s, m) * D + col * 4);
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    for (int mm = 0; mm < np; ++mm) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int col = lane + 32 * j;
+        if (col < vps) {
+          const uint4 x = stage[mm * vps + col];
+          const float f[4] = {__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z), __uint_as_float(x.w)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[j][q] = (m0 + mm == 0) ? f[q] : acc[j][q] + f[q];
+        }
+      }
+    }
+    __syncwarp();  // the next round overwrites the buffer
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int col = lane + 32 * j;
+    if (col < vps)
+      red_add4(table_grad + static_cast<int64_t>(key) * D + col * 4, acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
   }
 }
 
@@ -551,23 +625,38 @@ template <int L>
 __host__ __device__ constexpr int wide_warps() {
   return L >= 32 ? 2 : L >= 16 ? 4 : 8;  // about 33 KB of staging per block
 }
+constexpr int kWideTail = 64 * 4 + 48;  // per warp after the rows: 64 keys, 2 pending long runs, a count
+
 template <int L>
 __host__ __device__ constexpr size_t wide_smem() {
-  return static_cast<size_t>(wide_warps<L>()) * (kWideRows * L * 16 + 64 * 4);
+  return static_cast<size_t>(wide_warps<L>()) * (kWideRows * L * 16 + kWideTail);
+}
+
+struct PendingRun {
+  int64_t s;
+  int nc;
+  uint32_t key;
+};
+
+template <int L>
+__host__ __device__ constexpr int wide_min_blocks() {
+  return L <= 8 ? 4 : 6;  // keeps 8-warp blocks at <= 64 registers
 }
 
 template <int L, bool BF16>
-__global__ void __launch_bounds__(wide_warps<L>() * 32)
+__global__ void __launch_bounds__(wide_warps<L>() * 32, wide_min_blocks<L>())
 fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
                  const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
-                 int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
+                 const RunBook rb) {
   constexpr int RPI = 32 / L;         // rows per copy instruction = lane groups per warp
   constexpr int CPLN = BF16 ? 8 : 4;  // fp32 columns per lane
   extern __shared__ __align__(16) unsigned char wide_smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / L, sub = lane % L;
-  uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw) + warp * (kWideRows * L + 16);
+  uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw + warp * (kWideRows * L * 16 + kWideTail));
   uint32_t* keys_s = reinterpret_cast<uint32_t*>(rows_s + kWideRows * L);  // 64 keys
+  PendingRun* pend = reinterpret_cast<PendingRun*>(keys_s + 64);           // long runs this warp completed
+  int* npend = reinterpret_cast<int*>(pend + 2);
   const int64_t w = static_cast<int64_t>(blockIdx.x) * wide_warps<L>() + warp;
   wait_for_prior_grid();
   allow_next_grid();
@@ -578,6 +667,8 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
   keys_s[lane] = W.kA;
   keys_s[32 + lane] = W.kB;
+  if (lane == 0) *npend = 0;
+  __syncwarp();
 
   const uint64_t in_range = (W.b >= 64 ? ~0ull : ((1ull << W.b) - 1)) & ~((1ull << W.a) - 1);
   uint64_t rem = W.cm & in_range;  // chunk starts still to fold
@@ -616,19 +707,29 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
       const uint32_t key = keys_s[c];
       if (key == bad_key) continue;
       int64_t slot = 0;
-      const bool whole = chunk_is_whole_run(W, c, nxt, N, sub == 0, &slot, mc_len, mc_list, mc_count);
-      float* dst = (whole ? table_grad + static_cast<int64_t>(key) * D : csum + slot * D) + sub * CPLN;
-      if (whole) {
+      if (chunk_is_whole_run(W, c, nxt, N, &slot)) {
+        float* dst = table_grad + static_cast<int64_t>(key) * D + sub * CPLN;
 #pragma unroll
         for (int q = 0; q < CPLN; q += 4) red_add4(dst + q, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
       } else {
+        float* dst = csum + slot * D + sub * CPLN;
 #pragma unroll
         for (int q = 0; q < CPLN; q += 4)
           *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+        const unsigned gmask = L == 32 ? kFull : (((1u << L) - 1u) << (grp * L));
+        int64_t s = 0;
+        const int nc = chunk_stored(W, c, nxt, N, gmask, grp * L, rb, &s);
+        if (nc && sub == 0) {  // this chunk completed a long run: fold it once the window is done
+          const int at = atomicAdd(npend, 1);  // at most 2: a window holds chunks of at most 2 long runs
+          if (at < 2) pend[at] = PendingRun{s, nc, key};
+        }
       }
     }
     __syncwarp();  // the next round reuses the staging buffer
   }
+  const int n = min(*npend, 2);
+  for (int q = 0; q < n; ++q)
+    finish_run_staged(csum, pend[q].s, pend[q].nc, D, pend[q].key, table_grad, rows_s, kWideRows * L);
 }
 
 // Generic fold for row sizes the wide fold does not cover: lanes own
@@ -637,7 +738,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kFoldThreads, 3)
 fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, uint32_t bad_key,
                     const void* __restrict__ grad, int D, float* __restrict__ table_grad, float* __restrict__ csum,
-                    int* __restrict__ mc_len, int* __restrict__ mc_list, int* __restrict__ mc_count) {
+                    const RunBook rb) {
   constexpr int kBatch = 4;
   const int lane = threadIdx.x & 31;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5;
@@ -677,62 +778,33 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
           const uint32_t key = W.key_at(c);
           if (key != bad_key) {
             int64_t slot = 0;
-            if (chunk_is_whole_run(W, c, nxt, N, lane == 0, &slot, mc_len, mc_list, mc_count))
+            if (chunk_is_whole_run(W, c, nxt, N, &slot)) {
               red_add_row<0>(table_grad, key, D, acc);
-            else
+            } else {
               store_slot<0>(csum, slot, D, acc);
+              int64_t s = 0;
+              const int nc = chunk_stored(W, c, nxt, N, kFull, 0, rb, &s);
+              if (nc) {  // second level by the whole warp, lanes owning columns l, l+32, ...
+                Cols<0> sum;
+#pragma unroll
+                for (int q = 0; q < Cols<0>::n; ++q) {
+                  const int d = lane + 32 * q;
+                  sum.v[q] = d < D ? __ldcg(csum + chunk_slot(s, 0) * D + d) : 0.f;
+                }
+                for (int m = 1; m < nc; ++m) {
+#pragma unroll
+                  for (int q = 0; q < Cols<0>::n; ++q) {
+                    const int d = lane + 32 * q;
+                    if (d < D) sum.v[q] = sum.v[q] + __ldcg(csum + chunk_slot(s, m) * D + d);
+                  }
+                }
+                red_add_row<0>(table_grad, key, D, sum);
+              }
+            }
           }
         }
       }
     }
-  }
-}
-
-// Level 2: one warp per run longer than 32 hits folds the run's chunk sums in
-// order (loads issued kAhead at a time ahead of the adds); one final add into
-// table_grad.
-template <int CPL>
-__global__ void __launch_bounds__(kFoldThreads)
-fold_heavy_kernel(const uint32_t* __restrict__ K, int64_t N, uint32_t bad_key, const float* __restrict__ csum,
-                  const int* __restrict__ mc_len, const int* __restrict__ mc_list, const int* __restrict__ mc_count,
-                  int D, float* __restrict__ table_grad) {
-  constexpr int kAhead = CPL == 1 ? 32 : CPL == 2 ? 24 : CPL == 4 ? 16 : 8;
-  const int lane = threadIdx.x & 31;
-  wait_for_prior_grid();
-  const int count = *mc_count;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kFoldThreads / 32);
-  for (int64_t q = (static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x) >> 5; q < count; q += nwarps) {
-    const int64_t c0 = mc_list[q];
-    const int64_t len = min(static_cast<int64_t>(mc_len[c0 >> 5]), N - c0);  // clamp: never past the end
-    const int nc = static_cast<int>((len + kChunk - 1) / kChunk);
-    const uint32_t key = K[c0];
-    if (key >= bad_key) continue;
-    auto load_slot = [&](int64_t slot, Cols<CPL>& y) {
-      if constexpr (CPL == 0) {
-#pragma unroll
-        for (int k = 0; k < kMaxColsPerLane; ++k)
-          y.v[k] = (lane + 32 * k < D) ? csum[slot * D + lane + 32 * k] : 0.f;
-      } else {
-        const float* p = csum + slot * D + lane * CPL;
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) y.v[k] = p[k];
-      }
-    };
-    Cols<CPL> acc;
-    load_slot(2 * (c0 >> 5) + 1, acc);
-    for (int m0 = 1; m0 < nc; m0 += kAhead) {
-      Cols<CPL> y[kAhead];
-#pragma unroll
-      for (int u = 0; u < kAhead; ++u)
-        if (m0 + u < nc) load_slot(2 * ((c0 + static_cast<int64_t>(m0 + u) * kChunk) >> 5), y[u]);
-#pragma unroll
-      for (int u = 0; u < kAhead; ++u)
-        if (m0 + u < nc) {
-#pragma unroll
-          for (int k = 0; k < Cols<CPL>::n; ++k) acc.v[k] = acc.v[k] + y[u].v[k];
-        }
-    }
-    red_add_row<CPL>(table_grad, key, D, acc);
   }
 }
 
@@ -760,8 +832,8 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
 // host side
 // ---------------------------------------------------------------------------
 struct Layout {
-  size_t keys[2], vals[2], hist[2], off, total, csum, mc_len, mc_list, zeroed, total_bytes;
-  size_t zeroed_bytes;  // the sort's barrier counter and the heavy-run counter, cleared per call
+  size_t keys[2], vals[2], hist[2], off, total, csum, run_len, run_done, zeroed, total_bytes;
+  size_t zeroed_bytes;  // the sort's barrier counter (and a spare word), cleared per call
   int64_t nwin;
 };
 
@@ -783,8 +855,8 @@ Layout layout_for(int64_t N, int D) {
   L.off = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
   L.total = take(sizeof(uint32_t) * kRadix);
   L.csum = take(sizeof(float) * 2 * static_cast<size_t>(L.nwin) * D);
-  L.mc_len = take(sizeof(int) * L.nwin);
-  L.mc_list = take(sizeof(int) * L.nwin);
+  L.run_len = take(sizeof(int) * L.nwin);
+  L.run_done = take(sizeof(unsigned int) * L.nwin);
   L.zeroed_bytes = 2 * sizeof(unsigned int);
   L.zeroed = take(L.zeroed_bytes);
   L.total_bytes = off;
@@ -871,9 +943,11 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   sa.bar = reinterpret_cast<unsigned int*>(ws + L.zeroed);
   sa.status = status;
   float* csum = reinterpret_cast<float*>(ws + L.csum);
-  int* mc_len = reinterpret_cast<int*>(ws + L.mc_len);
-  int* mc_list = reinterpret_cast<int*>(ws + L.mc_list);
-  int* mc_count = reinterpret_cast<int*>(sa.bar + 1);
+  RunBook rb;
+  rb.len = reinterpret_cast<int*>(ws + L.run_len);
+  rb.done = reinterpret_cast<unsigned int*>(ws + L.run_done);
+  sa.run_done = rb.done;
+  sa.nwin = L.nwin;
 
   // key bits: keys lie in [0, num_rows] (num_rows marks a bad row)
   int bits = 0;
@@ -895,8 +969,7 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   const bool bf = gdt == PLE_BF16;
   const int lanes_per_row = static_cast<int>(static_cast<int64_t>(D) * (bf ? 2 : 4) / 16);
   auto fold = [&](auto kernel, dim3 grid, int threads, size_t smem) {
-    return launch_after(kernel, grid, dim3(threads), smem, s, Ks, Is, N, bad_key, grad, D, table_grad, csum,
-                        mc_len, mc_list, mc_count);
+    return launch_after(kernel, grid, dim3(threads), smem, s, Ks, Is, N, bad_key, grad, D, table_grad, csum, rb);
   };
 #define PLE_WIDE(LW, BF)                                                                                  \
   case 2 * LW + BF:                                                                                       \
@@ -913,19 +986,6 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   }
 #undef PLE_WIDE
   if (e != cudaSuccess) return cuda_fail(e);
-  const dim3 heavy_grid(static_cast<unsigned>(sm_count() * 4));
-  auto heavy = [&](auto kernel) {
-    return launch_after(kernel, heavy_grid, dim3(kFoldThreads), 0, s, Ks, N, bad_key,
-                        static_cast<const float*>(csum), static_cast<const int*>(mc_len),
-                        static_cast<const int*>(mc_list), static_cast<const int*>(mc_count), D, table_grad);
-  };
-  switch (cols_per_lane(D)) {
-    case 1: e = heavy(fold_heavy_kernel<1>); break;
-    case 2: e = heavy(fold_heavy_kernel<2>); break;
-    case 4: e = heavy(fold_heavy_kernel<4>); break;
-    case 8: e = heavy(fold_heavy_kernel<8>); break;
-    default: e = heavy(fold_heavy_kernel<0>); break;
-  }
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
