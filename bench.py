@@ -399,7 +399,7 @@ def main():
         table_host[uniq_rows.cpu().numpy()] = torch_to_np(table.index_select(0, uniq_rows))
         grad_host = torch_to_np(grad) if do_bwd else np.zeros((N, D), np.float32)
         tot_t, tot_s, reps = 0, 0.0, 0
-        while tot_s < args.cpu_seconds and reps < 50:
+        while tot_s < args.cpu_seconds and reps < 500:
             tt, dt = cpu_oracle_step(w, table_host, grad_host, threads)
             tot_t += tt
             tot_s += dt
