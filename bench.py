@@ -222,6 +222,8 @@ def main():
     ap.add_argument("--workload", default="single_layer_bf16")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--fwd-only", action="store_true", help="time the lookup alone (workloads marked fwd only)")
+    ap.add_argument("--slice", default=None, metavar="ROW_LEN:START:END",
+                    help="time the global-slice lookup of [START, END) of every ROW_LEN-token row (fwd only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=8192)
@@ -258,6 +260,13 @@ def main():
     w = workload(args.workload, replica_seed(args.seed, rank))
     plan = ple.Plan.from_workload(w)
     T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
+    sl = None
+    if args.slice:
+        row_len, s0, s1 = (int(x) for x in args.slice.split(":"))
+        if row_len < 1 or T % row_len or not (0 <= s0 < s1 <= row_len):
+            raise SystemExit("--slice needs ROW_LEN dividing the tokens and 0 <= START < END <= ROW_LEN")
+        sl = (row_len, s0, s1)
+        args.fwd_only = True
     tdt = torch.bfloat16 if w.table_dtype == 1 else torch.float32
     gdt = torch.bfloat16 if w.grad_dtype == 1 else torch.float32
     log(f"[rank {rank}] workload {w.name}: T={T} H={H} D={D} rows={w.num_rows} table {w.table_bytes / 1e9:.2f} GB")
@@ -266,8 +275,17 @@ def main():
     sgpu.fill_(table, w.table_seed, w.table_sigma)
     tokens = torch.from_numpy(w.tokens).to(dev)
     cu = torch.from_numpy(w.cu_seqlens).to(dev)
-    out = torch.empty(T, H, D, dtype=tdt, device=dev)
-    rows = torch.empty(T, H, dtype=torch.int64, device=dev)
+    T_out = T if sl is None else (T // sl[0]) * (sl[2] - sl[1])  # tokens looked up per step
+    out = torch.empty(T_out, H, D, dtype=tdt, device=dev)
+    rows = torch.empty(T_out, H, dtype=torch.int64, device=dev)
+
+    def lookup(tok_in, cu_in):
+        if sl is None:
+            ple.ple_lookup(plan, tok_in, cu_in, table, out=out, rows_out=rows)
+        else:
+            ple.ple_lookup_slice(plan, tok_in, cu_in, sl[0], sl[1], sl[2], table,
+                                 out=out.view(T // sl[0], sl[2] - sl[1], H, D),
+                                 rows_out=rows.view(T // sl[0], sl[2] - sl[1], H))
     do_bwd = not args.fwd_only
     if do_bwd:
         grad = torch.empty(N, D, dtype=gdt, device=dev)
@@ -283,7 +301,7 @@ def main():
         flush_r.sum()
 
     def step():
-        ple.ple_lookup(plan, tokens, cu, table, out=out, rows_out=rows)
+        lookup(tokens, cu)
         if do_bwd:
             ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
 
@@ -311,7 +329,7 @@ def main():
     for k in range(args.steps):
         flush_l2()                         # L2 flush between steps, outside the events
         ev[k][0].record(stream)
-        ple.ple_lookup(plan, tokens, cu, table, out=out, rows_out=rows)
+        lookup(tokens, cu)
         ev[k][1].record(stream)
         if do_bwd:
             ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
@@ -334,7 +352,8 @@ def main():
     peak, peak_kind = measured_peaks()
     e_t = 2 if w.table_dtype == 1 else 4
     e_g = 2 if w.grad_dtype == 1 else 4
-    fwd_bytes = 8 * T + 2 * N * D * e_t + 8 * N
+    N_out = T_out * H
+    fwd_bytes = 8 * T + 2 * N_out * D * e_t + 8 * N_out
     bwd_bytes = 8 * N + N * D * e_g + 2 * U * D * 4
     fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
     bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9 if do_bwd else None
@@ -358,14 +377,14 @@ def main():
             roofline = bwd_roof
 
     launches_per_step = 1 + (2 if do_bwd else 0)  # lookup_kernel; sort_kernel (all passes) and the fold kernel
-    value = world * T / (ms_step * 1e-3)
+    value = world * T_out / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers
     e2e = None
     if args.e2e_steps > 0:
         h_tok = torch.from_numpy(w.tokens).pin_memory()
         h_cu = torch.from_numpy(w.cu_seqlens).pin_memory()
-        h_out = torch.empty(T, H, D, dtype=tdt).pin_memory()
+        h_out = torch.empty(T_out, H, D, dtype=tdt).pin_memory()
         h_grad = grad.cpu().pin_memory() if do_bwd else None
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         d_tok, d_cu = torch.empty_like(tokens), torch.empty_like(cu)
@@ -376,7 +395,7 @@ def main():
             e0.record(stream)
             d_tok.copy_(h_tok, non_blocking=True)
             d_cu.copy_(h_cu, non_blocking=True)
-            ple.ple_lookup(plan, d_tok, d_cu, table, out=out, rows_out=rows)
+            lookup(d_tok, d_cu)
             if do_bwd:
                 d_grad.copy_(h_grad, non_blocking=True)
                 ple.ple_grad_scatter(plan, rows.view(-1), d_grad, table_grad, workspace=ws)
@@ -388,11 +407,11 @@ def main():
         (t_e2e_ms,) = reduce_max([statistics.mean(times)], dist, dev)
         h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
         e2e = {"value": world * T / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": N * D * e_t, "ms_per_step": t_e2e_ms,
+               "d2h_bytes_per_step": N_out * D * e_t, "ms_per_step": t_e2e_ms,
                "what": "pinned H2D tokens+cu_seqlens+grad_out, ple_lookup, ple_grad_scatter, D2H of the lookup output"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and sl is None:
         threads = os.cpu_count() or 1
         uniq_rows = torch.unique(rows)
         table_host = np.zeros((w.num_rows, D), np.uint16 if w.table_dtype == 1 else np.float32)
@@ -415,8 +434,10 @@ def main():
                 "vs_baseline": None, "dtype": "int64 hash, bf16 copy, f32 grad", "data": "synthetic",
                 "config": dict(describe(w), parallelism=f"replicas{world}",
                                l2="flushed between steps (512 MB written, then another 512 MB read); flush outside the step events",
-                               step="ple_lookup (rows saved) + ple_grad_scatter" if do_bwd else "ple_lookup"),
-                "fwd": {"ms": ms_fwd, "tokens_per_s": world * T / (ms_fwd * 1e-3), "gb_per_s": fwd_gbs,
+                               step=("ple_lookup (rows saved) + ple_grad_scatter" if do_bwd else
+                                     "ple_lookup" if sl is None else
+                                     f"ple_lookup_slice rows of {sl[0]}, positions [{sl[1]}, {sl[2]})")),
+                "fwd": {"ms": ms_fwd, "tokens_per_s": world * T_out / (ms_fwd * 1e-3), "gb_per_s": fwd_gbs,
                         "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "frac_of_measured": fwd_gbs / peak},
                 "bwd": None if not do_bwd else {
                     "ms": ms_bwd, "tokens_per_s": world * T / (ms_bwd * 1e-3), "gb_per_s": bwd_gbs,

@@ -31,7 +31,8 @@ PLE_BF16 = 1
 _DTYPES = {torch.float32: PLE_F32, torch.bfloat16: PLE_BF16}
 
 # every symbol include/ple.h declares
-EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_gather",
+EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_lookup_slice",
+           "ple_gather",
            "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic",
            "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_status",
            "ple_strerror", "ple_last_cuda_error")
@@ -71,6 +72,7 @@ def _lib():
         lib.ple_plan_num_heads.restype = i32
         lib.ple_hash.argtypes = [vp, vp, i64, vp, i32, vp, vp]
         lib.ple_lookup.argtypes = [vp, vp, i64, vp, i32, vp, vp, vp, vp]
+        lib.ple_lookup_slice.argtypes = [vp, vp, i64, vp, i32, i64, i64, i64, vp, vp, vp, vp]
         lib.ple_gather.argtypes = [vp, vp, i64, vp, vp, vp]
         lib.ple_grad_scatter_workspace_bytes.argtypes = [vp, i64]
         lib.ple_grad_scatter_workspace_bytes.restype = sz
@@ -83,7 +85,7 @@ def _lib():
         lib.ple_strerror.argtypes = [ctypes.c_int]
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
-        for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_gather", "ple_grad_scatter",
+        for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_lookup_slice", "ple_gather", "ple_grad_scatter",
                      "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_status",
                      "ple_last_cuda_error"):
             getattr(lib, name).restype = ctypes.c_int
@@ -182,6 +184,28 @@ def ple_lookup(plan: Plan, tokens, cu_seqlens, table, out=None, rows_out=None, s
         rows_out = torch.empty(T, plan.num_heads, dtype=torch.int64, device=tokens.device)
     _check(_lib().ple_lookup(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
                              _ptr(table), _ptr(out), _ptr(rows_out), _stream(tokens.device)), "ple_lookup")
+    return (out, rows_out) if rows_out is not None else out
+
+
+def ple_lookup_slice(plan: Plan, tokens, cu_seqlens, row_len: int, start: int, end: int, table, out=None,
+                     rows_out=None, save_rows: bool = False):
+    """Global-slice lookup: [B, end-start, H, D] values of positions
+    [start, end) of every row of row_len tokens, hashed with full context."""
+    _as_i64(tokens, "tokens")
+    _as_i32(cu_seqlens, "cu_seqlens")
+    if table.dtype != plan.table_dtype or not table.is_contiguous() or table.shape[-1] != plan.head_dim:
+        raise ValueError("table must be contiguous [num_rows, head_dim] in the plan's dtype")
+    T = tokens.numel()
+    if row_len < 1 or T % row_len != 0 or not (0 <= start <= end <= row_len):
+        raise ValueError("need num_tokens = B * row_len and 0 <= start <= end <= row_len")
+    B, W = T // row_len, end - start
+    if out is None:
+        out = torch.empty(B, W, plan.num_heads, plan.head_dim, dtype=table.dtype, device=table.device)
+    if rows_out is None and save_rows:
+        rows_out = torch.empty(B, W, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    _check(_lib().ple_lookup_slice(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, row_len,
+                                   start, end, _ptr(table), _ptr(out), _ptr(rows_out), _stream(tokens.device)),
+           "ple_lookup_slice")
     return (out, rows_out) if rows_out is not None else out
 
 

@@ -58,6 +58,29 @@ __device__ __forceinline__ void order_hashes(const HashParams& hp, const int64_t
   }
 }
 
+// Same order hashes for a lane whose token is not the next position after
+// the previous lane's (slices cross row boundaries): every preceding token is
+// loaded from global memory.
+__device__ __forceinline__ void order_hashes_direct(const HashParams& hp, const int64_t* __restrict__ tokens,
+                                                    const int32_t* __restrict__ cu, int32_t num_seqs, int64_t t,
+                                                    bool valid, int64_t (&hs)[kMaxOrder - 1]) {
+  const int64_t tok = valid ? tokens[t] : 0;
+  const int64_t seq_start = valid ? static_cast<int64_t>(cu[find_sequence(cu, num_seqs, t)]) : 0;
+  uint64_t h = static_cast<uint64_t>(tok) * static_cast<uint64_t>(hp.mults[0]);
+  bool keep = valid;
+#pragma unroll
+  for (int k = 1; k < kMaxOrder; ++k) {
+    if (k < hp.ngram_size) {
+      keep = keep && (t - k >= seq_start) && (t - k >= 0);
+      const int64_t prev = keep ? tokens[t - k] : 0;
+      keep = keep && (prev != hp.eos_id);
+      const int64_t ctx = keep ? prev : 0;
+      h += static_cast<uint64_t>(ctx) * static_cast<uint64_t>(hp.mults[k]);
+      hs[k - 1] = static_cast<int64_t>(h);
+    }
+  }
+}
+
 // rows of the tokens of this lane for every head, head j of order 2 + j/G.
 template <typename Emit>
 __device__ __forceinline__ void rows_of_token(const HashParams& hp, const HeadConst* consts,
@@ -145,12 +168,21 @@ __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ tabl
 // tokens, the warp turns the order hashes into TW*H row offsets in its own
 // slice of shared memory, then streams those rows.  Warps drift apart, so one
 // warp's hashing overlaps other warps' copies.
-template <int TW, int VL>
+// Output tokens of a lookup: all T packed tokens, or (global slice) for each
+// of the T / row_len rows the positions [start, start + width) of the row.
+struct OutMap {
+  int64_t count;    // output tokens
+  int64_t row_len;  // slice mode only
+  int64_t start;
+  int64_t width;
+};
+
+template <int TW, int VL, bool kSlice>
 __global__ void __launch_bounds__(kBlock, 4)
 lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
               const int32_t* __restrict__ cu, int32_t num_seqs, const unsigned char* __restrict__ table,
               int64_t num_rows, int32_t row_bytes, unsigned char* __restrict__ out,
-              int64_t* __restrict__ rows_out, unsigned int* status) {
+              int64_t* __restrict__ rows_out, const OutMap om, unsigned int* status) {
   static_assert(TW <= 32, "the first TW lanes hash the warp's tokens");
   extern __shared__ __align__(16) unsigned char smem[];
   const int H = hp.num_heads;
@@ -163,20 +195,26 @@ lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T
   check_seqlens(cu, num_seqs, T, status);
   __syncthreads();
 
-  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + warp) * TW;
-  if (t0 >= T) return;
+  const int64_t Tout = kSlice ? om.count : T;
+  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + warp) * TW;  // first output token
+  if (t0 >= Tout) return;
   {
-    const int64_t t = t0 + lane;
-    const bool valid = lane < TW && t < T;
+    const int64_t o = t0 + lane;
+    const bool valid = lane < TW && o < Tout;
     int64_t hs[kMaxOrder - 1];
-    order_hashes(hp, tokens, cu, num_seqs, t, valid, hs);
+    if constexpr (kSlice) {
+      const int64_t t = valid ? (o / om.width) * om.row_len + om.start + o % om.width : 0;
+      order_hashes_direct(hp, tokens, cu, num_seqs, t, valid, hs);
+    } else {
+      order_hashes(hp, tokens, cu, num_seqs, o, valid, hs);
+    }
     if (lane < TW) {
 #pragma unroll
       for (int m = 0; m < kMaxOrder - 1; ++m) hsh[lane * (kMaxOrder - 1) + m] = hs[m];
     }
   }
   __syncwarp();
-  const int ntok = static_cast<int>(min(static_cast<int64_t>(TW), T - t0));
+  const int ntok = static_cast<int>(min(static_cast<int64_t>(TW), Tout - t0));
   const int nhits = ntok * H;
   const int G = hp.heads_per_ngram;
   for (int q = lane; q < nhits; q += 32) {
@@ -220,16 +258,16 @@ int log2_exact(int v) {
   return -1;
 }
 
-template <int TW>
+template <int TW, bool kSlice>
 ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
-                           int32_t S, const void* table, void* out, int64_t* rows_out, unsigned int* status,
-                           cudaStream_t stream) {
+                           int32_t S, const void* table, void* out, int64_t* rows_out, const OutMap& om,
+                           unsigned int* status, cudaStream_t stream) {
   const int H = plan->hp.num_heads;
   constexpr int kWarps = kBlock / 32;
   const size_t smem = H * sizeof(HeadConst) + kWarps * TW * (kMaxOrder - 1) * sizeof(int64_t) +
                       static_cast<size_t>(kWarps) * TW * H * sizeof(int64_t);
   if (smem > 48 * 1024) return PLE_ERR_UNSUPPORTED;  // not reached: TW*H <= 512 keeps it under 48 KB
-  const int64_t warps = (T + TW - 1) / TW;
+  const int64_t warps = ((kSlice ? om.count : T) + TW - 1) / TW;
   const dim3 grid(static_cast<unsigned>((warps + kWarps - 1) / kWarps));
   const auto* tb = static_cast<const unsigned char*>(table);
   auto* ob = static_cast<unsigned char*>(out);
@@ -237,8 +275,8 @@ ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_
   const int64_t R = plan->num_rows;
 #define PLE_LOOKUP_CASE(VL)                                                                            \
   case VL:                                                                                             \
-    lookup_kernel<TW, VL><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,     \
-                                                          rows_out, status);                           \
+    lookup_kernel<TW, VL, kSlice><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob, \
+                                                                  rows_out, om, status);               \
     break;
   switch (log2_exact(rb >> 4)) {
     PLE_LOOKUP_CASE(0)
@@ -249,8 +287,8 @@ ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_
     PLE_LOOKUP_CASE(5)
     PLE_LOOKUP_CASE(6)
     default:
-      lookup_kernel<TW, -1><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
-                                                            rows_out, status);
+      lookup_kernel<TW, -1, kSlice><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
+                                                                    rows_out, om, status);
   }
 #undef PLE_LOOKUP_CASE
   return check_launch();
@@ -297,31 +335,66 @@ ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t T, 
   return check_launch();
 }
 
-ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
-                        int32_t S, const void* table, void* out, int64_t* rows_out, void* stream) {
-  ple_status_t st = check_hash_args(plan, tokens, T, cu, S);
-  if (st != PLE_OK || T == 0) return st;
-  if (table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
-  if (!aligned(table, 16) || !aligned(out, 16) || (rows_out != nullptr && !aligned(rows_out, 8)))
-    return PLE_ERR_ALIGNMENT;
+}  // extern "C"
+
+namespace {
+
+template <bool kSlice>
+ple_status_t dispatch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu, int32_t S,
+                             const void* table, void* out, int64_t* rows_out, const OutMap& om, void* stream) {
   cudaError_t e;
   unsigned int* status = status_word(&e);
   if (status == nullptr) return cuda_fail(e);
   const auto s = static_cast<cudaStream_t>(stream);
-  // tokens per warp: about 1-4K 16-byte vectors of copy work per warp, but
-  // enough warps to fill every SM several times over
+  const int64_t Tout = kSlice ? om.count : T;
+  // tokens per warp: at most about 1K 16-byte vectors of copy work per warp,
+  // and enough warps to fill every SM several times over
   const int64_t vec_per_token = static_cast<int64_t>(plan->hp.num_heads) * (plan->row_bytes >> 4);
   int tw = 32;
-  while (tw > 4 && (tw * vec_per_token > 4096 || (T + tw - 1) / tw < 32LL * sm_count())) tw >>= 1;
+  while (tw > 1 && (tw * vec_per_token > 1024 || (Tout + tw - 1) / tw < 32LL * sm_count())) tw >>= 1;
   while (tw > 1 && tw * plan->hp.num_heads > 512) tw >>= 1;  // row offsets of 8 warps stay <= 32 KB
   switch (tw) {
-    case 32: return launch_lookup<32>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-    case 16: return launch_lookup<16>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-    case 8: return launch_lookup<8>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-    case 4: return launch_lookup<4>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-    case 2: return launch_lookup<2>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
-    default: return launch_lookup<1>(plan, tokens, T, cu, S, table, out, rows_out, status, s);
+    case 32: return launch_lookup<32, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    case 16: return launch_lookup<16, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    case 8: return launch_lookup<8, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    case 4: return launch_lookup<4, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    case 2: return launch_lookup<2, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    default: return launch_lookup<1, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
   }
+}
+
+ple_status_t check_lookup_ptrs(const void* table, void* out, int64_t* rows_out) {
+  if (table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(table, 16) || !aligned(out, 16) || (rows_out != nullptr && !aligned(rows_out, 8)))
+    return PLE_ERR_ALIGNMENT;
+  return PLE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                        int32_t S, const void* table, void* out, int64_t* rows_out, void* stream) {
+  ple_status_t st = check_hash_args(plan, tokens, T, cu, S);
+  if (st != PLE_OK || T == 0) return st;
+  st = check_lookup_ptrs(table, out, rows_out);
+  if (st != PLE_OK) return st;
+  return dispatch_lookup<false>(plan, tokens, T, cu, S, table, out, rows_out, OutMap{T, T, 0, T}, stream);
+}
+
+ple_status_t ple_lookup_slice(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
+                              int32_t S, int64_t row_len, int64_t start, int64_t end, const void* table, void* out,
+                              int64_t* rows_out, void* stream) {
+  ple_status_t st = check_hash_args(plan, tokens, T, cu, S);
+  if (st != PLE_OK) return st;
+  if (row_len < 1 || T % row_len != 0 || start < 0 || start > end || end > row_len) return PLE_ERR_INVALID_ARG;
+  const int64_t count = (T / row_len) * (end - start);
+  if (count == 0) return PLE_OK;
+  st = check_lookup_ptrs(table, out, rows_out);
+  if (st != PLE_OK) return st;
+  return dispatch_lookup<true>(plan, tokens, T, cu, S, table, out, rows_out, OutMap{count, row_len, start,
+                                                                                    end - start}, stream);
 }
 
 ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* table, void* out,

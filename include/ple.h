@@ -110,6 +110,20 @@ ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t n
                         const int32_t* cu_seqlens, int32_t num_seqs, const void* table, void* out,
                         int64_t* rows_out, void* stream);
 
+/* Global-slice lookup (_forward_global_slice of Qwen3_8_FlashNextNGramEmbedding):
+ * the packed tokens are num_tokens / row_len rows of row_len tokens (a
+ * replicated [batch, global_sequence] batch); every row is hashed with its
+ * complete context (so a shard keeps the tokens before it and the EOS resets
+ * at its boundary), and only positions [start, end) of each row are looked
+ * up: out [B, end - start, H, head_dim], rows_out (nullable) [B, end - start, H].
+ * cu_seqlens describes the packed segments of the whole stream (they must not
+ * cross row boundaries for the rows to be independent).  Errors as
+ * ple_lookup, plus PLE_ERR_INVALID_ARG unless row_len >= 1 divides
+ * num_tokens and 0 <= start <= end <= row_len.  An empty slice is a no-op. */
+ple_status_t ple_lookup_slice(const ple_plan_t* plan, const int64_t* tokens, int64_t num_tokens,
+                              const int32_t* cu_seqlens, int32_t num_seqs, int64_t row_len, int64_t start,
+                              int64_t end, const void* table, void* out, int64_t* rows_out, void* stream);
+
 /* Gather precomputed rows (_lookup_ngram_ids): out[i, :] = table[rows[i], :]
  * for i < num_hits.  A row outside [0, num_rows) yields a zero output row
  * and the async PLE_ERR_BAD_ROW.  table and out 16-byte aligned. */

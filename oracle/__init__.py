@@ -113,6 +113,26 @@ def lookup(tokens, cu_seqlens, ngram_size, heads_per_ngram, eos_id, mults, prime
     return gather(r, table), r
 
 
+def slice_positions(num_tokens, row_len, start, end):
+    """Packed positions of the slice [start, end) of every row of row_len tokens."""
+    if row_len <= 0 or num_tokens % row_len != 0 or not (0 <= start <= end <= row_len):
+        raise ValueError("need num_tokens = B * row_len and 0 <= start <= end <= row_len")
+    B = num_tokens // row_len
+    return (np.arange(B)[:, None] * row_len + np.arange(start, end)[None, :]).reshape(-1)
+
+
+def lookup_slice(tokens, cu_seqlens, ngram_size, heads_per_ngram, eos_id, mults, primes, offsets, table,
+                 row_len, start, end):
+    """Global-slice lookup (NeMo engram API page, _forward_global_slice): hash
+    the complete packed stream, then gather only the slice [start, end) of
+    every row: values [B, end-start, H, D] and rows [B, end-start, H]."""
+    r = rows(tokens, cu_seqlens, ngram_size, heads_per_ngram, eos_id, mults, primes, offsets)
+    pos = slice_positions(len(tokens), row_len, start, end)
+    B = len(tokens) // row_len
+    sel = r[pos].reshape(B, end - start, r.shape[1])
+    return gather(sel, table), sel
+
+
 def _grad_args(grad):
     g = np.ascontiguousarray(grad)
     if g.dtype == np.float32:

@@ -102,6 +102,13 @@ def test_calls_reject_bad_arguments_on_host():
     assert lib.ple_grad_scatter(h, 0x1000, 2 ** 31, 0x2000, 1, 0x3000, 0x4000, 1 << 62, None) == \
         binding.PLE_ERR_UNSUPPORTED
     assert lib.ple_grad_scatter_atomic(h, None, 5, 0x2000, 1, 0x3000, None) == binding.PLE_ERR_INVALID_ARG
+    # global slice: row_len must divide num_tokens, 0 <= start <= end <= row_len; empty slice is a no-op
+    sl = lib.ple_lookup_slice
+    assert sl(h, 0x1000, 12, 0x1000, 1, 5, 0, 2, 0x3000, 0x4000, None, None) == binding.PLE_ERR_INVALID_ARG
+    assert sl(h, 0x1000, 12, 0x1000, 1, 4, 3, 2, 0x3000, 0x4000, None, None) == binding.PLE_ERR_INVALID_ARG
+    assert sl(h, 0x1000, 12, 0x1000, 1, 4, 0, 5, 0x3000, 0x4000, None, None) == binding.PLE_ERR_INVALID_ARG
+    assert sl(h, 0x1000, 12, 0x1000, 1, 4, 2, 2, 0x3000, 0x4000, None, None) == 0
+    assert sl(h, 0x1000, 12, 0x1000, 1, 4, 0, 2, 0x3008, 0x4000, None, None) == binding.PLE_ERR_ALIGNMENT
 
 
 def test_workspace_grows_with_hits():
@@ -116,6 +123,6 @@ def test_workspace_grows_with_hits():
 
 def test_strerror_covers_codes():
     lib = ple.lib()
-    for c in range(8):
+    for c in range(9):
         assert lib.ple_strerror(c)
     assert b"unknown" in lib.ple_strerror(99)

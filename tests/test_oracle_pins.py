@@ -331,3 +331,43 @@ def test_grad_single_final_add_and_negative_zero():
 def test_grad_rejects_out_of_range():
     with pytest.raises(ValueError):
         oracle.grad_apply(np.array([0, 9]), np.zeros((2, 4), np.float32), np.zeros((5, 4), np.float32))
+
+
+# ---------------------------------------------------------------------------
+# global-slice lookup
+# ---------------------------------------------------------------------------
+
+def test_slice_keeps_context_before_the_boundary():
+    """A shard [start, end) of a row hashes with the tokens before `start`
+    (the API page: hashing the full tensor preserves the preceding raw tokens
+    and EOS resets at a CP boundary): its first tokens differ from hashing the
+    shard's tokens alone, and equal the full rows restricted to the shard."""
+    rng = np.random.default_rng(21)
+    n, G = 3, 2
+    mults = synth.signed_mults(n, rng)
+    primes = synth.consecutive_primes(5003, (n - 1) * G)
+    offsets = synth.exclusive_prefix(primes)
+    row_len, B = 40, 3
+    tok = rng.integers(1, 50, row_len * B)
+    tok[row_len + 17] = 0  # an EOS just before the shard of row 1
+    cu = np.arange(0, row_len * B + 1, row_len)
+    table = rng.standard_normal((sum(primes), 8)).astype(np.float32)
+    vals, sel = oracle.lookup_slice(tok, cu, n, G, 0, mults, primes, offsets, table, row_len, 18, 30)
+    full = oracle.rows(tok, cu, n, G, 0, mults, primes, offsets).reshape(B, row_len, -1)
+    np.testing.assert_array_equal(sel, full[:, 18:30])
+    np.testing.assert_array_equal(vals, table[full[:, 18:30]])
+    alone = oracle.rows(tok[18:30], [0, 12], n, G, 0, mults, primes, offsets)
+    assert not np.array_equal(sel[0, :2], alone[:2])   # row 0: context from positions 16, 17
+    np.testing.assert_array_equal(sel[0, 2:], alone[2:])
+    # row 1: the EOS at position 17 resets the context, so its shard hashes as if alone
+    alone1 = oracle.rows(tok[row_len + 18:row_len + 30], [0, 12], n, G, 0, mults, primes, offsets)
+    np.testing.assert_array_equal(sel[1], alone1)
+
+
+def test_slice_bounds_rejected():
+    with pytest.raises(ValueError):
+        oracle.slice_positions(10, 4, 0, 2)
+    with pytest.raises(ValueError):
+        oracle.slice_positions(8, 4, 3, 2)
+    assert oracle.slice_positions(8, 4, 1, 3).tolist() == [1, 2, 5, 6]
+    assert oracle.slice_positions(8, 4, 2, 2).size == 0

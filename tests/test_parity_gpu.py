@@ -217,3 +217,27 @@ def test_library_loaded_from_tree(cuda_device):
     ple.lib()
     maps = open("/proc/self/maps").read()
     assert os.path.realpath(ple.binding.LIB_PATH) in maps
+
+
+@pytest.mark.parametrize("row_len,B,start,end", [(256, 1, 0, 256), (256, 1, 100, 180), (1000, 4, 333, 777),
+                                                 (64, 8, 0, 1), (64, 8, 63, 64), (300, 3, 17, 17)])
+def test_global_slice_lookup(cuda_device, row_len, B, start, end):
+    dev = cuda_device
+    rng = np.random.default_rng(row_len + start)
+    T = row_len * B
+    tok = rng.integers(0, 60, T)
+    tok[rng.random(T) < 0.05] = 0
+    # packed segments inside every row (a boundary at each row start, and one more per row)
+    cuts = sorted(set([b * row_len for b in range(B + 1)] + [b * row_len + row_len // 3 for b in range(B)]))
+    w = custom_workload("slice", tok, cuts, 4, 3, 0, synth.signed_mults(4, rng), synth.consecutive_primes(331, 9),
+                        40, synth.DTYPE_BF16)
+    plan = ple.Plan.from_workload(w)
+    host_table, table = small_table(w, dev)
+    out, rows = ple.ple_lookup_slice(plan, dev_i64(w.tokens, dev), dev_i32(w.cu_seqlens, dev), row_len, start, end,
+                                     table, save_rows=True)
+    assert ple.ple_status() == ple.PLE_OK
+    ref_vals, ref_rows = oracle.lookup_slice(w.tokens, w.cu_seqlens, w.ngram_size, w.heads_per_ngram, w.eos_id,
+                                             w.mults, w.primes, w.offsets, host_table, row_len, start, end)
+    assert out.shape == (B, end - start, w.num_heads, w.head_dim)
+    np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
+    np.testing.assert_array_equal(torch_to_values(out), ref_vals)
