@@ -56,6 +56,9 @@ def _load():
         lib.oracle_ple_gather.restype = ctypes.c_int
         lib.oracle_ple_gather_mt.argtypes = lib.oracle_ple_gather.argtypes + [ctypes.c_int32]
         lib.oracle_ple_gather_mt.restype = ctypes.c_int
+        lib.oracle_ple_gather_e4m3.argtypes = [_i64p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                               ctypes.c_int64, ctypes.c_void_p]
+        lib.oracle_ple_gather_e4m3.restype = ctypes.c_int
         lib.oracle_ple_count_unique.argtypes = [_i64p, ctypes.c_int64]
         lib.oracle_ple_count_unique.restype = ctypes.c_int64
         lib.oracle_ple_grad_sums.argtypes = [_i64p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int,
@@ -102,6 +105,19 @@ def gather(rows_, table: np.ndarray, threads: int = 1) -> np.ndarray:
     out = np.empty(r.shape + tab.shape[1:], dtype=tab.dtype)
     args = (_p(r, _i64p), r.size, tab.ctypes.data, tab.shape[0], row_bytes, out.ctypes.data)
     rc = _load().oracle_ple_gather(*args) if threads <= 1 else _load().oracle_ple_gather_mt(*args, threads)
+    if rc != 0:
+        raise ValueError("row outside the table")
+    return out
+
+
+def gather_e4m3(rows_, table_codes: np.ndarray) -> np.ndarray:
+    """Gather from an fp8 e4m3 table (uint8 codes [R, D]) widened to bf16
+    (uint16 bit patterns), shape rows.shape + [D]."""
+    r = np.ascontiguousarray(rows_, dtype=np.int64)
+    tab = np.ascontiguousarray(table_codes, dtype=np.uint8)
+    D = tab.shape[1]
+    out = np.empty(r.shape + (D,), dtype=np.uint16)
+    rc = _load().oracle_ple_gather_e4m3(_p(r, _i64p), r.size, tab.ctypes.data, tab.shape[0], D, out.ctypes.data)
     if rc != 0:
         raise ValueError("row outside the table")
     return out

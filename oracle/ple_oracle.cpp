@@ -185,6 +185,34 @@ int oracle_ple_gather_mt(const int64_t* rows, int64_t N, const void* table, int6
   return 0;
 }
 
+// bf16 bit pattern of an fp8 e4m3 code (OCP 8-bit floating point spec,
+// "E4M3": 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+// infinities, S.1111.111 is NaN).  Every e4m3 value is exactly a bf16 value.
+uint16_t e4m3_to_bf16_bits(uint8_t code) {
+  const uint16_t sign = static_cast<uint16_t>(code & 0x80) << 8;
+  const int e = (code >> 3) & 0xF, m = code & 0x7;
+  if (e == 0xF && m == 0x7) return sign | 0x7FC0;       // NaN
+  if (e == 0 && m == 0) return sign;                     // +-0
+  if (e == 0) {                                          // subnormal: m * 2^-9
+    int p = 2;
+    while (!((m >> p) & 1)) --p;                         // leading one of m
+    const int exp = p - 9 + 127;
+    const int frac = (m - (1 << p)) << (7 - p);
+    return sign | static_cast<uint16_t>(exp << 7) | static_cast<uint16_t>(frac);
+  }
+  return sign | static_cast<uint16_t>((e - 7 + 127) << 7) | static_cast<uint16_t>(m << 4);
+}
+
+// out[i, :] = bf16(table[rows[i], :]) for an fp8 e4m3 table [num_rows, D].
+int oracle_ple_gather_e4m3(const int64_t* rows, int64_t N, const uint8_t* table, int64_t num_rows, int64_t D,
+                           uint16_t* out) {
+  for (int64_t i = 0; i < N; ++i)
+    if (rows[i] < 0 || rows[i] >= num_rows) return -1;
+  for (int64_t i = 0; i < N; ++i)
+    for (int64_t d = 0; d < D; ++d) out[i * D + d] = e4m3_to_bf16_bits(table[rows[i] * D + d]);
+  return 0;
+}
+
 // Number of distinct rows among rows[0..N).
 int64_t oracle_ple_count_unique(const int64_t* rows, int64_t N) {
   std::vector<int64_t> r(rows, rows + N);

@@ -40,6 +40,7 @@ IH4_SD = math.sqrt((65536.0 ** 2 - 1.0) / 3.0)
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
+DTYPE_E4M3 = 2  # fp8 e4m3 codes: uniform random finite codes (8 per counter output)
 
 
 def value_scale(sigma: float) -> np.float32:
@@ -82,8 +83,21 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def counter_e4m3(seed: int, idx: np.ndarray) -> np.ndarray:
+    """fp8 e4m3 codes: byte (i mod 8) of u(seed, i div 8); the two NaN codes
+    (x.1111.111) become the largest finite code of their sign."""
+    idx = np.asarray(idx, dtype=np.uint64)
+    u = counter_u64(seed, idx // np.uint64(8))
+    code = ((u >> (np.uint64(8) * (idx % np.uint64(8)))) & np.uint64(0xFF)).astype(np.uint8)
+    nan = (code & 0x7F) == 0x7F
+    code[nan] ^= 0x01
+    return code
+
+
 def counter_values(seed: int, idx: np.ndarray, sigma: float, dtype: int) -> np.ndarray:
-    """Values as stored: fp32 array, or bf16 bit patterns as uint16."""
+    """Values as stored: fp32 array, bf16 bit patterns as uint16, or fp8 codes as uint8."""
+    if dtype == DTYPE_E4M3:
+        return counter_e4m3(seed, idx)
     v = counter_f32(seed, idx, sigma)
     if dtype == DTYPE_F32:
         return v
@@ -259,7 +273,7 @@ class Workload:
 
     @property
     def table_elem_bytes(self) -> int:
-        return 4 if self.table_dtype == DTYPE_F32 else 2
+        return {DTYPE_F32: 4, DTYPE_BF16: 2, DTYPE_E4M3: 1}[self.table_dtype]
 
     @property
     def grad_elem_bytes(self) -> int:
@@ -320,6 +334,15 @@ def single_layer_bf16(seed: int = 0, total: int = 32768) -> Workload:
                     offsets, R, 64, DTYPE_BF16, seed + 101, 0.02, DTYPE_BF16, seed + 202, 1.0)
 
 
+def large_table_fp8(seed: int = 0, total: int = 65536) -> Workload:
+    """The large-table workload with the table stored as fp8 e4m3 (the pages'
+    checkpoint format): 25.8 GB, rows widened to bf16 by the lookup."""
+    w = large_table(seed, total)
+    w.name = "large_table_fp8"
+    w.table_dtype = DTYPE_E4M3
+    return w
+
+
 def large_table(seed: int = 0, total: int = 65536) -> Workload:
     """65536 packed tokens (lengths 1k-8k), Zipf(1.1), n=4, 8 heads per order
     (24 heads), 24 consecutive primes >= 8,400,000 (~2.0e8 rows), D=128 bf16
@@ -347,6 +370,7 @@ def backward_stress(seed: int = 0, total: int = 131072) -> Workload:
 def sweep_point(tokens: int = 131072, head_dim: int = 128, ngram_size: int = 3, heads_per_ngram: int = 8,
                 table_gb: float = 16.0, ids: str = "zipf", seed: int = 0,
                 table_dtype: int = DTYPE_BF16) -> Workload:
+    # (an fp8 table: table_dtype=DTYPE_E4M3)
     """One point of the sweep: per-head primes are consecutive primes >=
     table_bytes / (elem * D * H), so the table holds about ``table_gb`` GB."""
     rng, lens = _packed_stream(tokens, 1024, 8192, seed)
@@ -358,10 +382,10 @@ def sweep_point(tokens: int = 131072, head_dim: int = 128, ngram_size: int = 3, 
         raise ValueError(ids)
     tok = inject_eos(tok, 0.005, 0, rng)
     H = (ngram_size - 1) * heads_per_ngram
-    elem = 4 if table_dtype == DTYPE_F32 else 2
+    elem = {DTYPE_F32: 4, DTYPE_BF16: 2, DTYPE_E4M3: 1}[table_dtype]
     per_head = max(3, int(table_gb * 1e9 / (elem * head_dim * H)))
     mults, primes, offsets, R = _hash_constants(ngram_size, heads_per_ngram, per_head, rng)
-    name = f"sweep_T{tokens}_D{head_dim}_n{ngram_size}_{ids}_{table_gb:g}GB"
+    name = f"sweep_T{tokens}_D{head_dim}_n{ngram_size}_{ids}_{table_gb:g}GB" + ("_fp8" if table_dtype == DTYPE_E4M3 else "")
     return Workload(name, tok, cu_seqlens_from_lengths(lens), ngram_size, heads_per_ngram, 0, mults,
                     primes, offsets, R, head_dim, table_dtype, seed + 101, 0.02, DTYPE_BF16, seed + 202, 1.0)
 
@@ -371,4 +395,5 @@ WORKLOADS = {
     "single_layer_bf16": single_layer_bf16,
     "large_table": large_table,
     "backward_stress": backward_stress,
+    "large_table_fp8": large_table_fp8,
 }

@@ -62,12 +62,41 @@ __global__ void fill_bf16(uint64_t state0, uint64_t count, float k, uint16_t* __
     dst[i] = (uint16_t)bf16_bits(value_f32(state0, i, k));
 }
 
+// fp8 e4m3 codes: byte (i mod 8) of u(seed, i / 8), NaN codes moved to the
+// largest finite code of their sign; each thread writes 16 codes.
+__global__ void fill_e4m3(uint64_t state0, uint64_t count, unsigned char* __restrict__ dst) {
+  const uint64_t nvec = count / 16;
+  for (uint64_t v = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; v < nvec;
+       v += (uint64_t)gridDim.x * blockDim.x) {
+    uint32_t w[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint64_t u = sm64_out(state0, v * 2 + half);
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const uint32_t byte = (u >> (8 * b)) & 0xFF;
+        if ((byte & 0x7F) == 0x7F) u ^= (1ull << (8 * b));
+      }
+      w[half * 2] = (uint32_t)u;
+      w[half * 2 + 1] = (uint32_t)(u >> 32);
+    }
+    reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  for (uint64_t i = nvec * 16 + blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < count;
+       i += (uint64_t)gridDim.x * blockDim.x) {
+    uint32_t byte = (sm64_out(state0, i / 8) >> (8 * (i % 8))) & 0xFF;
+    if ((byte & 0x7F) == 0x7F) byte ^= 1u;
+    dst[i] = (unsigned char)byte;
+  }
+}
+
 }  // namespace
 
 extern "C" {
 
 // Fill dst[0..count) with the generator's values for indices 0..count-1.
-// dtype 0 = fp32, 1 = bf16 (bit patterns).  dst must be 16-byte aligned.
+// dtype 0 = fp32, 1 = bf16 (bit patterns), 2 = fp8 e4m3 codes.  dst must be
+// 16-byte aligned.
 // Returns 0 on success, else the cudaError_t of the launch.
 int synth_fill(uint64_t seed, uint64_t count, float k, int dtype, void* dst, cudaStream_t stream) {
   if (count == 0) return 0;
@@ -81,6 +110,8 @@ int synth_fill(uint64_t seed, uint64_t count, float k, int dtype, void* dst, cud
     fill_f32<<<grid, 256, 0, stream>>>(state0, count, k, static_cast<float*>(dst));
   else if (dtype == 1)
     fill_bf16<<<grid, 256, 0, stream>>>(state0, count, k, static_cast<uint16_t*>(dst));
+  else if (dtype == 2)
+    fill_e4m3<<<grid, 256, 0, stream>>>(state0, count, static_cast<unsigned char*>(dst));
   else
     return -2;
   return (int)cudaGetLastError();

@@ -10,7 +10,7 @@ import ctypes
 import os
 import subprocess
 
-from . import DTYPE_BF16, DTYPE_F32, value_scale
+from . import DTYPE_BF16, DTYPE_E4M3, DTYPE_F32, value_scale
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsynth_fill.so")
@@ -41,7 +41,7 @@ def _load():
 
 
 def fill_(tensor, seed: int, sigma: float) -> None:
-    """Fill a contiguous fp32 or bf16 CUDA tensor with generator values."""
+    """Fill a contiguous fp32, bf16 or fp8 e4m3 CUDA tensor with generator values."""
     import torch
 
     if not tensor.is_cuda or not tensor.is_contiguous():
@@ -50,6 +50,8 @@ def fill_(tensor, seed: int, sigma: float) -> None:
         code = DTYPE_F32
     elif tensor.dtype == torch.bfloat16:
         code = DTYPE_BF16
+    elif tensor.dtype == torch.float8_e4m3fn:
+        code = DTYPE_E4M3
     else:
         raise ValueError(f"unsupported dtype {tensor.dtype}")
     stream = torch.cuda.current_stream(tensor.device).cuda_stream

@@ -371,3 +371,28 @@ def test_slice_bounds_rejected():
         oracle.slice_positions(8, 4, 3, 2)
     assert oracle.slice_positions(8, 4, 1, 3).tolist() == [1, 2, 5, 6]
     assert oracle.slice_positions(8, 4, 2, 2).size == 0
+
+
+# ---------------------------------------------------------------------------
+# fp8 e4m3 table widening
+# ---------------------------------------------------------------------------
+
+def test_e4m3_widening_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8).reshape(16, 16)
+    got = oracle.gather_e4m3(np.arange(16), codes)  # [16, 16] bf16 bits
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float32)
+    ref_bits = ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    finite = ~torch.isnan(ref).numpy()
+    np.testing.assert_array_equal(got[finite], ref_bits[finite])
+    # the two NaN codes stay NaN, with their sign
+    nan_got = synth.bf16_bits_to_f32(got[~finite])
+    assert np.all(np.isnan(nan_got)) and (~finite).sum() == 2
+    # exactness: bf16 -> fp32 equals torch's fp8 -> fp32 on every finite code
+    np.testing.assert_array_equal(synth.bf16_bits_to_f32(got[finite]), ref.numpy()[finite])
+
+
+def test_e4m3_spot_values():
+    table = np.array([[0x38, 0x7E, 0x01, 0x80, 0xB8, 0x08, 0x07, 0x00] * 2], np.uint8)
+    v = synth.bf16_bits_to_f32(oracle.gather_e4m3(np.array([0]), table))[0, :8]
+    assert v.tolist() == [1.0, 448.0, 2.0 ** -9, -0.0, -1.0, 2.0 ** -6, 7 * 2.0 ** -9, 0.0]
+    assert np.signbit(v[3])
