@@ -58,16 +58,21 @@ def workload(name: str, seed: int):
     if name.startswith("sweep:"):
         kw = dict(kv.split("=") for kv in name[len("sweep:"):].split(",") if kv)
         conv = {"tokens": int, "head_dim": int, "ngram_size": int, "heads_per_ngram": int, "table_gb": float,
-                "ids": str}
+                "ids": str, "table_dtype": lambda v: {"f32": 0, "bf16": 1, "e4m3": 2}[v]}
         return synth.sweep_point(seed=seed, **{k: conv[k](v) for k, v in kw.items()})
     raise SystemExit(f"unknown workload {name}")
+
+
+DTYPE_NAMES = {0: "f32", 1: "bf16", 2: "e4m3"}
+ELEM_BYTES = {0: 4, 1: 2, 2: 1}
+HOST_DTYPE = {0: np.float32, 1: np.uint16, 2: np.uint8}  # the generator's host representation
 
 
 def describe(w):
     return {"workload": w.name, "tokens": w.num_tokens, "sequences": int(len(w.cu_seqlens) - 1),
             "ngram_size": w.ngram_size, "heads_per_ngram": w.heads_per_ngram, "heads": w.num_heads,
             "head_dim": w.head_dim, "table_rows": w.num_rows,
-            "table_dtype": "bf16" if w.table_dtype == 1 else "f32",
+            "table_dtype": DTYPE_NAMES[w.table_dtype],
             "table_gb": round(w.table_bytes / 1e9, 3), "grad_dtype": "bf16" if w.grad_dtype == 1 else "f32"}
 
 
@@ -167,7 +172,10 @@ def cpu_oracle_step(w, table_host, grad_host, threads, tokens_limit=None):
     t0 = time.perf_counter()
     rows = oracle.rows(tok, cu.astype(np.int32), w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
                        w.offsets, threads=threads)
-    oracle.gather(rows, table_host, threads=threads)
+    if w.table_dtype == 2:
+        oracle.gather_e4m3(rows, table_host)
+    else:
+        oracle.gather(rows, table_host, threads=threads)
     oracle.grad_sums(rows, grad_host[: rows.size], threads=threads)
     return T, time.perf_counter() - t0
 
@@ -189,7 +197,7 @@ def run_reference(args, rank, world):
                          w.mults, w.primes, w.offsets)
     # a full-size host table whose touched rows hold the generated values
     # (np.zeros pages stay unbacked until written, so untouched rows cost no RAM)
-    table_host = np.zeros((w.num_rows, w.head_dim), np.uint16 if w.table_dtype == 1 else np.float32)
+    table_host = np.zeros((w.num_rows, w.head_dim), HOST_DTYPE[w.table_dtype])
     uniq = np.unique(rows_s)
     table_host[uniq] = w.table_rows(uniq)
     grad_host = synth.dense_values(w.grad_seed, rows_s.size * w.head_dim, w.grad_sigma,
@@ -267,7 +275,8 @@ def main():
             raise SystemExit("--slice needs ROW_LEN dividing the tokens and 0 <= START < END <= ROW_LEN")
         sl = (row_len, s0, s1)
         args.fwd_only = True
-    tdt = torch.bfloat16 if w.table_dtype == 1 else torch.float32
+    tdt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float8_e4m3fn}[w.table_dtype]
+    odt = plan.out_dtype  # bf16 for an fp8 table
     gdt = torch.bfloat16 if w.grad_dtype == 1 else torch.float32
     log(f"[rank {rank}] workload {w.name}: T={T} H={H} D={D} rows={w.num_rows} table {w.table_bytes / 1e9:.2f} GB")
 
@@ -276,7 +285,7 @@ def main():
     tokens = torch.from_numpy(w.tokens).to(dev)
     cu = torch.from_numpy(w.cu_seqlens).to(dev)
     T_out = T if sl is None else (T // sl[0]) * (sl[2] - sl[1])  # tokens looked up per step
-    out = torch.empty(T_out, H, D, dtype=tdt, device=dev)
+    out = torch.empty(T_out, H, D, dtype=odt, device=dev)
     rows = torch.empty(T_out, H, dtype=torch.int64, device=dev)
 
     def lookup(tok_in, cu_in):
@@ -350,10 +359,11 @@ def main():
                                           statistics.mean(bwd_ms)], dist, dev)
 
     peak, peak_kind = measured_peaks()
-    e_t = 2 if w.table_dtype == 1 else 4
+    e_t = ELEM_BYTES[w.table_dtype]
+    e_o = out.element_size()
     e_g = 2 if w.grad_dtype == 1 else 4
     N_out = T_out * H
-    fwd_bytes = 8 * T + 2 * N_out * D * e_t + 8 * N_out
+    fwd_bytes = 8 * T + N_out * D * (e_t + e_o) + 8 * N_out
     bwd_bytes = 8 * N + N * D * e_g + 2 * U * D * 4
     fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
     bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9 if do_bwd else None
@@ -384,7 +394,7 @@ def main():
     if args.e2e_steps > 0:
         h_tok = torch.from_numpy(w.tokens).pin_memory()
         h_cu = torch.from_numpy(w.cu_seqlens).pin_memory()
-        h_out = torch.empty(T_out, H, D, dtype=tdt).pin_memory()
+        h_out = torch.empty(T_out, H, D, dtype=odt).pin_memory()
         h_grad = grad.cpu().pin_memory() if do_bwd else None
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         d_tok, d_cu = torch.empty_like(tokens), torch.empty_like(cu)
@@ -407,15 +417,16 @@ def main():
         (t_e2e_ms,) = reduce_max([statistics.mean(times)], dist, dev)
         h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
         e2e = {"value": world * T / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": N_out * D * e_t, "ms_per_step": t_e2e_ms,
+               "d2h_bytes_per_step": N_out * D * e_o, "ms_per_step": t_e2e_ms,
                "what": "pinned H2D tokens+cu_seqlens+grad_out, ple_lookup, ple_grad_scatter, D2H of the lookup output"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and sl is None:
         threads = os.cpu_count() or 1
         uniq_rows = torch.unique(rows)
-        table_host = np.zeros((w.num_rows, D), np.uint16 if w.table_dtype == 1 else np.float32)
-        table_host[uniq_rows.cpu().numpy()] = torch_to_np(table.index_select(0, uniq_rows))
+        table_host = np.zeros((w.num_rows, D), HOST_DTYPE[w.table_dtype])
+        raw = table.view(torch.uint8) if w.table_dtype == 2 else table
+        table_host[uniq_rows.cpu().numpy()] = torch_to_np(raw.index_select(0, uniq_rows))
         grad_host = torch_to_np(grad) if do_bwd else np.zeros((N, D), np.float32)
         tot_t, tot_s, reps = 0, 0.0, 0
         while tot_s < args.cpu_seconds and reps < 500:
@@ -431,7 +442,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "int64 hash, bf16 copy, f32 grad", "data": "synthetic",
+                "vs_baseline": None, "dtype": ("int64 hash, e4m3->bf16 widening copy, f32 grad" if w.table_dtype == 2 else
+                          f"int64 hash, {DTYPE_NAMES[w.table_dtype]} copy, f32 grad"), "data": "synthetic",
                 "config": dict(describe(w), parallelism=f"replicas{world}",
                                l2="flushed between steps (512 MB written, then another 512 MB read); flush outside the step events",
                                step=("ple_lookup (rows saved) + ple_grad_scatter" if do_bwd else

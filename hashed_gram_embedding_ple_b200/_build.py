@@ -4,6 +4,7 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -30,11 +31,18 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
-    cmd = ["nvcc", "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared", "-Xcompiler", "-fPIC,-Wall",
-           f"-I{INCLUDE}", "-o", LIB_PATH, *[os.path.join(CSRC, s) for s in SOURCES]]
+    flags = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC,-Wall", f"-I{INCLUDE}"]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+        flags.append("-Xptxas=-v")
+    with tempfile.TemporaryDirectory(prefix="ple_build_") as tmp:
+        # one nvcc per translation unit, run side by side, then one link
+        objs = [os.path.join(tmp, os.path.splitext(s)[0] + ".o") for s in SOURCES]
+        procs = [subprocess.Popen(["nvcc", *flags, "-c", "-o", o, os.path.join(CSRC, s)])
+                 for s, o in zip(SOURCES, objs)]
+        codes = [p.wait() for p in procs]
+        if any(codes):
+            raise subprocess.CalledProcessError(max(codes), "nvcc")
+        subprocess.run(["nvcc", *ARCH, "-shared", "-o", LIB_PATH, *objs], check=True)
     return LIB_PATH
 
 

@@ -27,8 +27,11 @@ PLE_ERR_TIMEOUT = 8
 
 PLE_F32 = 0
 PLE_BF16 = 1
+PLE_F8E4M3 = 2
 
-_DTYPES = {torch.float32: PLE_F32, torch.bfloat16: PLE_BF16}
+_DTYPES = {torch.float32: PLE_F32, torch.bfloat16: PLE_BF16}          # tables and gradients
+_TABLE_DTYPES = {**_DTYPES, torch.float8_e4m3fn: PLE_F8E4M3}           # tables only
+_DTYPE_OF_CODE = {PLE_F32: torch.float32, PLE_BF16: torch.bfloat16, PLE_F8E4M3: torch.float8_e4m3fn}
 
 # every symbol include/ple.h declares
 EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_lookup_slice",
@@ -122,20 +125,22 @@ class Plan:
         self._offsets = (ctypes.c_int64 * max(1, len(offsets)))(*[int(o) for o in offsets])
         if len(mults) != ngram_size or len(primes) != H or len(offsets) != H:
             raise ValueError("mults must have ngram_size entries; primes and offsets (ngram_size-1)*heads_per_ngram")
-        if table_dtype not in _DTYPES:
-            raise ValueError(f"table dtype must be float32 or bfloat16, not {table_dtype}")
+        if table_dtype not in _TABLE_DTYPES:
+            raise ValueError(f"table dtype must be float32, bfloat16 or float8_e4m3fn, not {table_dtype}")
         p = _Params(ngram_size, heads_per_ngram, int(eos_id), self._mults, self._primes, self._offsets,
-                    int(num_rows), int(head_dim), _DTYPES[table_dtype])
+                    int(num_rows), int(head_dim), _TABLE_DTYPES[table_dtype])
         handle = ctypes.c_void_p()
         _check(_lib().ple_plan_create(ctypes.byref(p), ctypes.byref(handle)), "ple_plan_create")
         self._h = handle
         self.ngram_size, self.heads_per_ngram, self.num_heads = ngram_size, heads_per_ngram, H
         self.num_rows, self.head_dim, self.table_dtype = int(num_rows), int(head_dim), table_dtype
+        # lookups of an fp8 table are widened to bf16
+        self.out_dtype = torch.bfloat16 if table_dtype == torch.float8_e4m3fn else table_dtype
 
     @classmethod
     def from_workload(cls, w):
         return cls(w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes, w.offsets, w.num_rows,
-                   w.head_dim, torch.float32 if w.table_dtype == PLE_F32 else torch.bfloat16)
+                   w.head_dim, _DTYPE_OF_CODE[w.table_dtype])
 
     @property
     def handle(self):
@@ -158,6 +163,33 @@ def _as_i32(t, name):
         raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
 
 
+def _check_table(plan: Plan, table):
+    if table.dtype != plan.table_dtype or not table.is_contiguous() or table.shape[-1] != plan.head_dim \
+            or table.numel() != plan.num_rows * plan.head_dim or not table.is_cuda:
+        raise ValueError("table must be a contiguous CUDA tensor [num_rows, head_dim] in the plan's dtype")
+
+
+def _out(plan: Plan, out, shape, device):
+    """The caller's output tensor, checked, or a new one."""
+    if out is None:
+        return torch.empty(*shape, dtype=plan.out_dtype, device=device)
+    n = 1
+    for d in shape:
+        n *= d
+    if out.dtype != plan.out_dtype or not out.is_contiguous() or out.numel() != n or out.device != device:
+        raise ValueError(f"out must be a contiguous {plan.out_dtype} tensor of {n} elements on {device}")
+    return out
+
+
+def _rows(rows, shape, device):
+    n = 1
+    for d in shape:
+        n *= d
+    if rows.dtype != torch.int64 or not rows.is_contiguous() or rows.numel() != n or rows.device != device:
+        raise ValueError(f"rows_out must be a contiguous int64 tensor of {n} elements on {device}")
+    return rows
+
+
 def ple_hash(plan: Plan, tokens, cu_seqlens, rows=None):
     """int64 [T, H] global rows of every (token, head)."""
     _as_i64(tokens, "tokens")
@@ -165,23 +197,26 @@ def ple_hash(plan: Plan, tokens, cu_seqlens, rows=None):
     T = tokens.numel()
     if rows is None:
         rows = torch.empty(T, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    else:
+        _rows(rows, (T, plan.num_heads), tokens.device)
     _check(_lib().ple_hash(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, _ptr(rows),
                            _stream(tokens.device)), "ple_hash")
     return rows
 
 
 def ple_lookup(plan: Plan, tokens, cu_seqlens, table, out=None, rows_out=None, save_rows: bool = False):
-    """Hash fused with the gather: [T, H, D] values in the table dtype.
-    With save_rows (or a rows_out tensor) also returns the [T, H] rows."""
+    """Hash fused with the gather: [T, H, D] values in the table dtype (bf16
+    for an fp8 table).  With save_rows (or a rows_out tensor) also returns the
+    [T, H] rows."""
     _as_i64(tokens, "tokens")
     _as_i32(cu_seqlens, "cu_seqlens")
-    if table.dtype != plan.table_dtype or not table.is_contiguous() or table.shape[-1] != plan.head_dim:
-        raise ValueError("table must be contiguous [num_rows, head_dim] in the plan's dtype")
+    _check_table(plan, table)
     T = tokens.numel()
-    if out is None:
-        out = torch.empty(T, plan.num_heads, plan.head_dim, dtype=table.dtype, device=table.device)
+    out = _out(plan, out, (T, plan.num_heads, plan.head_dim), table.device)
     if rows_out is None and save_rows:
         rows_out = torch.empty(T, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    elif rows_out is not None:
+        _rows(rows_out, (T, plan.num_heads), tokens.device)
     _check(_lib().ple_lookup(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
                              _ptr(table), _ptr(out), _ptr(rows_out), _stream(tokens.device)), "ple_lookup")
     return (out, rows_out) if rows_out is not None else out
@@ -193,16 +228,16 @@ def ple_lookup_slice(plan: Plan, tokens, cu_seqlens, row_len: int, start: int, e
     [start, end) of every row of row_len tokens, hashed with full context."""
     _as_i64(tokens, "tokens")
     _as_i32(cu_seqlens, "cu_seqlens")
-    if table.dtype != plan.table_dtype or not table.is_contiguous() or table.shape[-1] != plan.head_dim:
-        raise ValueError("table must be contiguous [num_rows, head_dim] in the plan's dtype")
+    _check_table(plan, table)
     T = tokens.numel()
     if row_len < 1 or T % row_len != 0 or not (0 <= start <= end <= row_len):
         raise ValueError("need num_tokens = B * row_len and 0 <= start <= end <= row_len")
     B, W = T // row_len, end - start
-    if out is None:
-        out = torch.empty(B, W, plan.num_heads, plan.head_dim, dtype=table.dtype, device=table.device)
+    out = _out(plan, out, (B, W, plan.num_heads, plan.head_dim), table.device)
     if rows_out is None and save_rows:
         rows_out = torch.empty(B, W, plan.num_heads, dtype=torch.int64, device=tokens.device)
+    elif rows_out is not None:
+        _rows(rows_out, (B, W, plan.num_heads), tokens.device)
     _check(_lib().ple_lookup_slice(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1, row_len,
                                    start, end, _ptr(table), _ptr(out), _ptr(rows_out), _stream(tokens.device)),
            "ple_lookup_slice")
@@ -210,12 +245,11 @@ def ple_lookup_slice(plan: Plan, tokens, cu_seqlens, row_len: int, start: int, e
 
 
 def ple_gather(plan: Plan, rows, table, out=None):
-    """out[i] = table[rows[i]] for flat rows; shape rows.shape + [D]."""
+    """out[i] = table[rows[i]] for flat rows; shape rows.shape + [D] (bf16
+    for an fp8 table)."""
     _as_i64(rows, "rows")
-    if table.dtype != plan.table_dtype or not table.is_contiguous():
-        raise ValueError("table must be contiguous in the plan's dtype")
-    if out is None:
-        out = torch.empty(*rows.shape, plan.head_dim, dtype=table.dtype, device=table.device)
+    _check_table(plan, table)
+    out = _out(plan, out, (*rows.shape, plan.head_dim), table.device)
     _check(_lib().ple_gather(plan.handle, _ptr(rows), rows.numel(), _ptr(table), _ptr(out),
                              _stream(rows.device)), "ple_gather")
     return out
@@ -236,12 +270,17 @@ def _grad_dtype(g):
     return _DTYPES[g.dtype]
 
 
+def _check_table_grad(plan: Plan, table_grad):
+    if table_grad.dtype != torch.float32 or not table_grad.is_contiguous() or not table_grad.is_cuda \
+            or table_grad.numel() != plan.num_rows * plan.head_dim:
+        raise ValueError("table_grad must be a contiguous float32 CUDA tensor [num_rows, head_dim]")
+
+
 def ple_grad_scatter(plan: Plan, rows, grad_out, table_grad, workspace=None):
     """Deterministic table_grad += per-row sums of grad_out (fixed chunked order)."""
     _as_i64(rows, "rows")
     gdt = _grad_dtype(grad_out)
-    if table_grad.dtype != torch.float32 or not table_grad.is_contiguous():
-        raise ValueError("table_grad must be contiguous float32")
+    _check_table_grad(plan, table_grad)
     N = rows.numel()
     if grad_out.numel() != N * plan.head_dim:
         raise ValueError("grad_out must hold num_hits * head_dim values")
@@ -256,6 +295,7 @@ def ple_grad_scatter_atomic(plan: Plan, rows, grad_out, table_grad):
     """Non-deterministic fp32 atomic variant (speed reference)."""
     _as_i64(rows, "rows")
     gdt = _grad_dtype(grad_out)
+    _check_table_grad(plan, table_grad)
     N = rows.numel()
     if grad_out.numel() != N * plan.head_dim:
         raise ValueError("grad_out must hold num_hits * head_dim values")
@@ -270,8 +310,7 @@ def ple_grad_scatter_noalloc(plan: Plan, rows, grad_out, table_grad):
     rules on overlapping calls."""
     _as_i64(rows, "rows")
     gdt = _grad_dtype(grad_out)
-    if table_grad.dtype != torch.float32 or not table_grad.is_contiguous():
-        raise ValueError("table_grad must be contiguous float32")
+    _check_table_grad(plan, table_grad)
     N = rows.numel()
     if grad_out.numel() != N * plan.head_dim:
         raise ValueError("grad_out must hold num_hits * head_dim values")

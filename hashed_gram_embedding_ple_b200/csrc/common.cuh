@@ -57,6 +57,12 @@ __device__ __forceinline__ uint4 ld_nc_na(const void* p) {
 }
 
 // 16-byte streaming store (evict-first: the output is not re-read here).
+__device__ __forceinline__ uint2 ld_nc_na8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ void st_cs(void* p, const uint4& v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)

@@ -8,7 +8,8 @@
 // output is column (q mod V) of hit (q div V), V = row_bytes / 16, so the
 // stores of a warp are contiguous and each row is read by V consecutive
 // lanes.  UNROLL independent loads are in flight per thread before the
-// matching stores are issued.
+// matching stores are issued.  An fp8 E4M3 table is widened to bf16 on the
+// way (8 bytes of codes in, 16 bytes of bf16 out per unit).
 #include "common.cuh"
 
 namespace ple {
@@ -135,7 +136,7 @@ hash_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
 // ---------------------------------------------------------------------------
 // Row streaming shared by the fused lookup and the gather: `lanes` threads
 // (a warp or a block) copy nhits rows, vector q of the output being column
-// q mod V of hit q div V.
+// q mod V of hit q div V (V = row bytes / 16).
 // ---------------------------------------------------------------------------
 template <int VL, int kLanes>
 __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ table,
@@ -163,6 +164,92 @@ __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ tabl
   }
 }
 
+// E4M3 -> bf16 widening, two codes per 32-bit word, on the integer and
+// bf16x2 pipes.  For a code c = S.EEEE.MMM the pattern S.0000EEEE.MMM0000
+// read as bf16 is (-1)^S 2^(E-127) (1 + M/8) for E > 0 and the subnormal
+// (-1)^S (M/8) 2^-126 for E = 0; one exact bf16 multiply by 2^120 turns both
+// into the E4M3 value (bias 7: 2^(E-7) (1 + M/8), and M 2^-9).  The two NaN
+// codes S.1111.111 would come out as +-480; they are patched to S | 0x7FC0.
+constexpr uint32_t kBf16x2Two120 = 0x7B807B80u;  // {2^120, 2^120}
+
+__device__ __forceinline__ uint32_t e4m3_pair_to_bf16x2(uint32_t codes4, int pair) {
+  // a = {c_lo, c_hi} in the low byte of each half; b = the same in the high byte
+  const uint32_t a = __byte_perm(codes4, 0, pair ? 0x4342 : 0x4140);
+  const uint32_t b = __byte_perm(codes4, 0, pair ? 0x3424 : 0x1404);
+  const uint32_t x = ((a << 4) & 0x07F007F0u) | (b & 0x80008000u);
+  uint32_t y;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(kBf16x2Two120));
+  return y;
+}
+
+// The NaN patch of one pair (rare path).
+__device__ __noinline__ uint32_t e4m3_pair_nan_patch(uint32_t codes4, int pair, uint32_t y) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t c = (codes4 >> (16 * pair + 8 * h)) & 0xFFu;
+    if ((c & 0x7Fu) == 0x7Fu) y = (y & (0xFFFF0000u >> (16 * h))) | ((((c & 0x80u) << 8) | 0x7FC0u) << (16 * h));
+  }
+  return y;
+}
+
+// Eight codes to eight bf16 values (one 16-byte store).
+__device__ __forceinline__ uint4 widen8(const uint2 c) {
+  uint4 o = make_uint4(e4m3_pair_to_bf16x2(c.x, 0), e4m3_pair_to_bf16x2(c.x, 1), e4m3_pair_to_bf16x2(c.y, 0),
+                       e4m3_pair_to_bf16x2(c.y, 1));
+  // a byte b with (b & 0x7F) == 0x7F becomes 0x80 after +1 on its low 7 bits
+  const uint32_t nan = (((c.x & 0x7F7F7F7Fu) + 0x01010101u) | ((c.y & 0x7F7F7F7Fu) + 0x01010101u)) & 0x80808080u;
+  if (nan != 0) {
+    o.x = e4m3_pair_nan_patch(c.x, 0, o.x);
+    o.y = e4m3_pair_nan_patch(c.x, 1, o.y);
+    o.z = e4m3_pair_nan_patch(c.y, 0, o.z);
+    o.w = e4m3_pair_nan_patch(c.y, 1, o.w);
+  }
+  return o;
+}
+
+// Widening variant of copy_hits for an E4M3 table: the unit is 8 bytes of
+// codes (V8 = row bytes / 8 per row) and becomes one 16-byte bf16 store at
+// byte 16 q of the output, so the stores of a warp stay contiguous.  Twice
+// as many units as vectors: twice the unroll keeps the bytes in flight.
+constexpr int kWidenUnroll = 2 * kUnroll;
+
+template <int VL, int kLanes>
+__device__ __forceinline__ void widen_hits(const unsigned char* __restrict__ table,
+                                           const int64_t* __restrict__ rowoff, int nhits, int v_rt,
+                                           unsigned char* __restrict__ out, int tid) {
+  constexpr int VL8 = VL >= 0 ? VL + 1 : -1;
+  const int V = VL8 >= 0 ? (1 << VL8) : 2 * v_rt;
+  const int total = nhits * V;
+  for (int base = tid; base < total; base += kLanes * kWidenUnroll) {
+    uint2 v[kWidenUnroll];
+#pragma unroll
+    for (int u = 0; u < kWidenUnroll; ++u) {
+      const int q = base + u * kLanes;
+      if (q < total) {
+        const int hit = VL8 >= 0 ? (q >> VL8) : q / V;
+        const int col = q - hit * V;
+        const int64_t off = rowoff[hit];
+        v[u] = off >= 0 ? ld_nc_na8(table + off + col * 8) : make_uint2(0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kWidenUnroll; ++u) {
+      const int q = base + u * kLanes;
+      if (q < total) st_cs(out + static_cast<int64_t>(q) * 16, widen8(v[u]));
+    }
+  }
+}
+
+template <int VL, int kLanes, bool kWiden>
+__device__ __forceinline__ void stream_hits(const unsigned char* __restrict__ table,
+                                            const int64_t* __restrict__ rowoff, int nhits, int v_rt,
+                                            unsigned char* __restrict__ out, int tid) {
+  if constexpr (kWiden)
+    widen_hits<VL, kLanes>(table, rowoff, nhits, v_rt, out, tid);
+  else
+    copy_hits<VL, kLanes>(table, rowoff, nhits, v_rt, out, tid);
+}
+
 // Fused lookup.  Every warp owns TW consecutive tokens and works alone (no
 // block barrier after the constants are staged): its first TW lanes hash the
 // tokens, the warp turns the order hashes into TW*H row offsets in its own
@@ -177,7 +264,7 @@ struct OutMap {
   int64_t width;
 };
 
-template <int TW, int VL, bool kSlice>
+template <int TW, int VL, bool kSlice, bool kWiden>
 __global__ void __launch_bounds__(kBlock, 4)
 lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T,
               const int32_t* __restrict__ cu, int32_t num_seqs, const unsigned char* __restrict__ table,
@@ -227,12 +314,13 @@ lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T
     if (rows_out != nullptr) rows_out[t0 * H + q] = row;
   }
   __syncwarp();
-  copy_hits<VL, 32>(table, rowoff, nhits, row_bytes >> 4, out + t0 * H * row_bytes, lane);
+  const int64_t out_row_bytes = static_cast<int64_t>(row_bytes) * (kWiden ? 2 : 1);
+  stream_hits<VL, 32, kWiden>(table, rowoff, nhits, row_bytes >> 4, out + t0 * H * out_row_bytes, lane);
 }
 
 constexpr int kGatherHits = 512;  // hits per block of the plain gather
 
-template <int VL>
+template <int VL, bool kWiden>
 __global__ void __launch_bounds__(kBlock, 4)
 gather_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows,
               const unsigned char* __restrict__ table, int32_t row_bytes, unsigned char* __restrict__ out,
@@ -249,7 +337,8 @@ gather_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows,
   }
   if (bad) raise_flag(status, PLE_ERR_BAD_ROW);
   __syncthreads();
-  copy_hits<VL, kBlock>(table, rowoff, nh, row_bytes >> 4, out + h0 * row_bytes, threadIdx.x);
+  const int64_t out_row_bytes = static_cast<int64_t>(row_bytes) * (kWiden ? 2 : 1);
+  stream_hits<VL, kBlock, kWiden>(table, rowoff, nh, row_bytes >> 4, out + h0 * out_row_bytes, threadIdx.x);
 }
 
 int log2_exact(int v) {
@@ -258,7 +347,7 @@ int log2_exact(int v) {
   return -1;
 }
 
-template <int TW, bool kSlice>
+template <int TW, bool kSlice, bool kWiden>
 ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu,
                            int32_t S, const void* table, void* out, int64_t* rows_out, const OutMap& om,
                            unsigned int* status, cudaStream_t stream) {
@@ -275,8 +364,8 @@ ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_
   const int64_t R = plan->num_rows;
 #define PLE_LOOKUP_CASE(VL)                                                                            \
   case VL:                                                                                             \
-    lookup_kernel<TW, VL, kSlice><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob, \
-                                                                  rows_out, om, status);               \
+    lookup_kernel<TW, VL, kSlice, kWiden><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, \
+                                                                          rb, ob, rows_out, om, status);     \
     break;
   switch (log2_exact(rb >> 4)) {
     PLE_LOOKUP_CASE(0)
@@ -287,8 +376,8 @@ ple_status_t launch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_
     PLE_LOOKUP_CASE(5)
     PLE_LOOKUP_CASE(6)
     default:
-      lookup_kernel<TW, -1, kSlice><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb, ob,
-                                                                    rows_out, om, status);
+      lookup_kernel<TW, -1, kSlice, kWiden><<<grid, kBlock, smem, stream>>>(plan->hp, tokens, T, cu, S, tb, R, rb,
+                                                                            ob, rows_out, om, status);
   }
 #undef PLE_LOOKUP_CASE
   return check_launch();
@@ -353,14 +442,22 @@ ple_status_t dispatch_lookup(const ple_plan_t* plan, const int64_t* tokens, int6
   int tw = 32;
   while (tw > 1 && (tw * vec_per_token > 1024 || (Tout + tw - 1) / tw < 32LL * sm_count())) tw >>= 1;
   while (tw > 1 && tw * plan->hp.num_heads > 512) tw >>= 1;  // row offsets of 8 warps stay <= 32 KB
+  const bool widen = plan->table_dtype == PLE_F8E4M3;
+#define PLE_TW_CASE(TWV)                                                                                      \
+  case TWV:                                                                                                   \
+    return widen ? launch_lookup<TWV, kSlice, true>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s) \
+                 : launch_lookup<TWV, kSlice, false>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
   switch (tw) {
-    case 32: return launch_lookup<32, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
-    case 16: return launch_lookup<16, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
-    case 8: return launch_lookup<8, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
-    case 4: return launch_lookup<4, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
-    case 2: return launch_lookup<2, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
-    default: return launch_lookup<1, kSlice>(plan, tokens, T, cu, S, table, out, rows_out, om, status, s);
+    PLE_TW_CASE(32)
+    PLE_TW_CASE(16)
+    PLE_TW_CASE(8)
+    PLE_TW_CASE(4)
+    PLE_TW_CASE(2)
+    PLE_TW_CASE(1)
+    default:
+      return PLE_ERR_UNSUPPORTED;  // not reached: tw is a power of two in 1..32
   }
+#undef PLE_TW_CASE
 }
 
 ple_status_t check_lookup_ptrs(const void* table, void* out, int64_t* rows_out) {
@@ -412,9 +509,13 @@ ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, 
   auto* ob = static_cast<unsigned char*>(out);
   const int rb = plan->row_bytes;
   const int64_t R = plan->num_rows;
-#define PLE_GATHER_CASE(VL)                                                       \
-  case VL:                                                                        \
-    gather_kernel<VL><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);    \
+  const bool widen = plan->table_dtype == PLE_F8E4M3;
+#define PLE_GATHER_CASE(VL)                                                                   \
+  case VL:                                                                                    \
+    if (widen)                                                                                \
+      gather_kernel<VL, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);        \
+    else                                                                                      \
+      gather_kernel<VL, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);       \
     break;
   switch (log2_exact(rb >> 4)) {
     PLE_GATHER_CASE(0)
@@ -425,7 +526,10 @@ ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, 
     PLE_GATHER_CASE(5)
     PLE_GATHER_CASE(6)
     default:
-      gather_kernel<-1><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
+      if (widen)
+        gather_kernel<-1, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
+      else
+        gather_kernel<-1, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
   }
 #undef PLE_GATHER_CASE
   return check_launch();

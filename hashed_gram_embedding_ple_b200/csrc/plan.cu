@@ -82,8 +82,9 @@ ple_status_t ple_plan_create(const ple_params_t* p, ple_plan_t** out) {
   const int64_t H = static_cast<int64_t>(p->ngram_size - 1) * p->heads_per_ngram;
   if (H > ple::kMaxHeads) return PLE_ERR_UNSUPPORTED;
   if (p->num_rows < 1 || p->head_dim < 1) return PLE_ERR_INVALID_ARG;
-  if (p->table_dtype != PLE_F32 && p->table_dtype != PLE_BF16) return PLE_ERR_INVALID_ARG;
-  const int64_t elem = p->table_dtype == PLE_F32 ? 4 : 2;
+  if (p->table_dtype != PLE_F32 && p->table_dtype != PLE_BF16 && p->table_dtype != PLE_F8E4M3)
+    return PLE_ERR_INVALID_ARG;
+  const int64_t elem = p->table_dtype == PLE_F32 ? 4 : p->table_dtype == PLE_BF16 ? 2 : 1;
   const int64_t row_bytes = elem * p->head_dim;
   if (row_bytes % 16 != 0) return PLE_ERR_ALIGNMENT;
   if (row_bytes > (1 << 20)) return PLE_ERR_UNSUPPORTED;

@@ -61,7 +61,15 @@ typedef enum {
   PLE_ERR_TIMEOUT = 8        /* async: a bounded wait between the blocks of a kernel ran out */
 } ple_status_t;
 
-typedef enum { PLE_F32 = 0, PLE_BF16 = 1 } ple_dtype_t;
+/* Element types.  PLE_F8E4M3 is a table type only: OCP FP8 E4M3 codes
+ * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities,
+ * S.1111.111 is NaN): the official checkpoint's weights are FP8 ("Feat/qwen38
+ * flash next" pull request, Summary), and no scale format is given there, so
+ * the codes are widened unscaled.  A lookup of such a table
+ * writes bf16: every finite E4M3 value is exactly a bf16 value, so the
+ * widening is exact; a NaN code gives the quiet bf16 NaN with the code's
+ * sign (0x7FC0 or 0xFFC0). */
+typedef enum { PLE_F32 = 0, PLE_BF16 = 1, PLE_F8E4M3 = 2 } ple_dtype_t;
 
 /* Hash and table description (constructor parameters of
  * Qwen3_8_FlashNextNGramEmbedding and Qwen3_8_FlashNextEngramTableConfig). */
@@ -74,7 +82,8 @@ typedef struct {
   const int64_t* offsets;   /* HOST [H] first global row of each head */
   int64_t num_rows;         /* table rows; every [offset, offset+prime) inside, disjoint */
   int32_t head_dim;         /* values per row, D */
-  ple_dtype_t table_dtype;  /* element type of the table and of lookup output */
+  ple_dtype_t table_dtype;  /* element type of the table; lookup output is the same
+                               type, except bf16 for a PLE_F8E4M3 table */
 } ple_params_t;
 
 typedef struct ple_plan ple_plan_t;
@@ -102,8 +111,8 @@ ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t num
 
 /* Hash fused with the gather (forward of Qwen3_8_FlashNextNGramEmbedding):
  * out[t, j, :] = table[row[t, j], :], out [num_tokens, H, head_dim] in the
- * table dtype (= [tokens, H * head_dim] with heads concatenated).  The copy
- * is exact.  rows_out, if not NULL, receives the int64 [num_tokens, H] rows
+ * table dtype, bf16 for an E4M3 table (= [tokens, H * head_dim] with heads
+ * concatenated).  The copy (and the E4M3 widening) is exact.  rows_out, if not NULL, receives the int64 [num_tokens, H] rows
  * (to feed ple_grad_scatter).  table and out must be 16-byte aligned.
  * Errors as ple_hash. */
 ple_status_t ple_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t num_tokens,
@@ -125,8 +134,9 @@ ple_status_t ple_lookup_slice(const ple_plan_t* plan, const int64_t* tokens, int
                               int64_t end, const void* table, void* out, int64_t* rows_out, void* stream);
 
 /* Gather precomputed rows (_lookup_ngram_ids): out[i, :] = table[rows[i], :]
- * for i < num_hits.  A row outside [0, num_rows) yields a zero output row
- * and the async PLE_ERR_BAD_ROW.  table and out 16-byte aligned. */
+ * for i < num_hits, out in the lookup's output type (bf16 for an E4M3
+ * table).  A row outside [0, num_rows) yields a zero output row and the
+ * async PLE_ERR_BAD_ROW.  table and out 16-byte aligned. */
 ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits, const void* table,
                         void* out, void* stream);
 
@@ -145,7 +155,7 @@ size_t ple_grad_scatter_workspace_bytes(const ple_plan_t* plan, int64_t num_hits
  * it for a fresh gradient).  Hits whose row is outside [0, num_rows) are
  * dropped and raise the async PLE_ERR_BAD_ROW.  table_grad and grad_out
  * 16-byte aligned; workspace 256-byte aligned.  Errors: PLE_ERR_WORKSPACE,
- * PLE_ERR_UNSUPPORTED (num_rows >= 2^32 - 1 or num_hits >= 2^31),
+ * PLE_ERR_UNSUPPORTED (head_dim > 256, num_rows >= 2^32 - 1 or num_hits >= 2^31),
  * PLE_ERR_INVALID_ARG, PLE_ERR_ALIGNMENT, PLE_ERR_CUDA. */
 ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits,
                               const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,

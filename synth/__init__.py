@@ -370,9 +370,9 @@ def backward_stress(seed: int = 0, total: int = 131072) -> Workload:
 def sweep_point(tokens: int = 131072, head_dim: int = 128, ngram_size: int = 3, heads_per_ngram: int = 8,
                 table_gb: float = 16.0, ids: str = "zipf", seed: int = 0,
                 table_dtype: int = DTYPE_BF16) -> Workload:
-    # (an fp8 table: table_dtype=DTYPE_E4M3)
     """One point of the sweep: per-head primes are consecutive primes >=
-    table_bytes / (elem * D * H), so the table holds about ``table_gb`` GB."""
+    table_bytes / (elem * D * H), so the table holds about ``table_gb`` GB
+    (table_dtype=DTYPE_E4M3 for an fp8 table)."""
     rng, lens = _packed_stream(tokens, 1024, 8192, seed)
     if ids == "zipf":
         tok = zipf_ids(tokens, 1.1, VOCAB, rng)

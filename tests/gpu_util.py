@@ -13,18 +13,27 @@ def dev_i32(a, device):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
 
 
+TORCH_DTYPE = {synth.DTYPE_F32: torch.float32, synth.DTYPE_BF16: torch.bfloat16,
+               synth.DTYPE_E4M3: torch.float8_e4m3fn}
+
+
 def values_to_torch(v: np.ndarray, dtype_code: int) -> torch.Tensor:
-    """Host generator output (fp32, or bf16 bits as uint16) as a CPU tensor."""
+    """Host generator output (fp32, bf16 bits as uint16 or fp8 codes as
+    uint8) as a CPU tensor."""
     if dtype_code == synth.DTYPE_F32:
         return torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+    if dtype_code == synth.DTYPE_E4M3:
+        return torch.from_numpy(np.ascontiguousarray(v, dtype=np.uint8)).view(torch.float8_e4m3fn)
     return torch.from_numpy(np.ascontiguousarray(v, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
 
 
 def torch_to_values(t: torch.Tensor) -> np.ndarray:
-    """Device tensor back to the host representation (fp32, or bf16 bits)."""
+    """Device tensor back to the host representation (fp32, bf16 bits or fp8 codes)."""
     t = t.detach().cpu().contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
 
 
@@ -39,8 +48,7 @@ def device_table(w, device):
     """Table generated on the device by the twin generator (large workloads)."""
     from synth import gpu as sgpu
 
-    dt = torch.float32 if w.table_dtype == synth.DTYPE_F32 else torch.bfloat16
-    t = torch.empty(w.num_rows, w.head_dim, dtype=dt, device=device)
+    t = torch.empty(w.num_rows, w.head_dim, dtype=TORCH_DTYPE[w.table_dtype], device=device)
     sgpu.fill_(t, w.table_seed, w.table_sigma)
     return t
 

@@ -44,6 +44,10 @@ def _plan(**kw):
 def test_plan_accepts_valid():
     p = _plan()
     assert ple.lib().ple_plan_num_heads(p.handle) == 4
+    q = _plan(head_dim=16, table_dtype=binding.torch.float8_e4m3fn)  # 16 codes = one 16-byte vector
+    assert q.out_dtype == binding.torch.bfloat16
+    with pytest.raises(ValueError):
+        _plan(table_dtype=binding.torch.float16)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -56,6 +60,7 @@ def test_plan_accepts_valid():
     (dict(offsets=[-1, 7, 18, 31]), binding.PLE_ERR_INVALID_ARG),
     (dict(primes=[7, 11, 13, 2 ** 62 + 1], num_rows=2 ** 63 - 1), binding.PLE_ERR_INVALID_ARG),
     (dict(head_dim=4), binding.PLE_ERR_ALIGNMENT),                          # 8-byte rows
+    (dict(head_dim=8, table_dtype=binding.torch.float8_e4m3fn), binding.PLE_ERR_ALIGNMENT),  # 8 fp8 codes
     (dict(head_dim=0), binding.PLE_ERR_INVALID_ARG),
     (dict(heads_per_ngram=33, mults=[1, 2, 3], primes=[5] * 66, offsets=[0] * 66), binding.PLE_ERR_UNSUPPORTED),
 ])

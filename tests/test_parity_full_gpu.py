@@ -41,7 +41,8 @@ def check_forward_full(w, dev, samples=8192):
     # input check: the device generator wrote the host generator's values
     rng = np.random.default_rng(7)
     probe = rng.integers(0, w.num_rows, 64)
-    np.testing.assert_array_equal(torch_to_values(table[dev_i64(probe, dev)]), w.table_rows(probe))
+    raw = table.view(torch.uint8) if table.dtype == torch.float8_e4m3fn else table
+    np.testing.assert_array_equal(torch_to_values(raw[dev_i64(probe, dev)]), w.table_rows(probe))
 
     tok, cu = dev_i64(w.tokens, dev), dev_i32(w.cu_seqlens, dev)
     out, rows = ple.ple_lookup(plan, tok, cu, table, save_rows=True)
@@ -56,9 +57,15 @@ def check_forward_full(w, dev, samples=8192):
     sel = ref_rows.reshape(-1)[hits]
     uniq, inv = np.unique(sel, return_inverse=True)
     compact = w.table_rows(uniq)
-    np.testing.assert_array_equal(got, oracle.gather(inv, compact))
-    # every hit against torch's gather of the same table
-    ref_all = torch.nn.functional.embedding(rows.view(-1), table)
+    fp8 = w.table_dtype == synth.DTYPE_E4M3
+    np.testing.assert_array_equal(got, oracle.gather_e4m3(inv, compact) if fp8 else oracle.gather(inv, compact))
+    # every hit against torch's gather of the same table (and, for fp8 codes,
+    # torch's own widening of the gathered codes; the generator draws no NaN code)
+    if fp8:
+        ref_all = table.view(torch.uint8).index_select(0, rows.view(-1)).view(torch.float8_e4m3fn)
+        ref_all = ref_all.to(torch.bfloat16)
+    else:
+        ref_all = torch.nn.functional.embedding(rows.view(-1), table)
     assert torch.equal(_bits(out.view(-1, w.head_dim)), _bits(ref_all))
     del ref_all
     del table, out, flat
@@ -98,6 +105,12 @@ def test_large_table_full(cuda_device):
     check_forward_full(w, cuda_device)
 
 
+def test_large_table_fp8_full(cuda_device):
+    w = synth.large_table_fp8(0)
+    assert w.table_bytes > 25e9
+    check_forward_full(w, cuda_device)
+
+
 def test_backward_stress_full(cuda_device):
     w = synth.backward_stress(0)
     plan = ple.Plan.from_workload(w)
@@ -114,6 +127,7 @@ def test_backward_stress_full(cuda_device):
     dict(tokens=1 << 20, head_dim=32, ngram_size=2, ids="uniform", table_gb=16.0),
     dict(tokens=16384, head_dim=256, ngram_size=4, ids="zipf", table_gb=2.0),
     dict(tokens=131072, head_dim=128, ngram_size=3, ids="zipf", table_gb=80.0),
+    dict(tokens=131072, head_dim=128, ngram_size=3, ids="zipf", table_gb=16.0, table_dtype=synth.DTYPE_E4M3),
 ])
 def test_sweep_points(cuda_device, kw):
     w = synth.sweep_point(**kw)
