@@ -10,9 +10,11 @@
 //   added once into table_grad[r].
 //
 // Pipeline (all in the caller's workspace, no allocation):
-//   1. sort_kernel (cooperative): 32-bit keys from the int64 rows (bad rows
-//      -> key R), LSD radix sort with 8-bit digits, stable, values = hit index;
-//   2. fold kernel: one warp per window of 32 sorted positions; it folds the
+//   1. key_hist_kernel: 32-bit keys from the int64 rows (bad rows -> key R)
+//      and the digit counts of every radix pass;
+//   2. sort_pass_kernel, once per 8-bit digit: LSD radix sort, stable,
+//      values = hit index (tiles find their offsets by look-back);
+//   3. fold kernel: one warp per window of 32 sorted positions; it folds the
 //      chunks that start in its window (a chunk start is a position whose
 //      offset from its run's first position is a multiple of 32), adds a
 //      whole single-chunk run into table_grad, or stores the chunk sum of a
@@ -41,27 +43,38 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // ---------------------------------------------------------------------------
-// radix sort: one cooperative kernel runs every pass
+// radix sort: LSD, 8-bit digits, stable, one kernel per pass
 //
-// All blocks of the grid are resident at once (cooperative launch), so the
-// phases of a pass are separated by a grid barrier instead of kernel
-// boundaries.  Block b owns the contiguous positions [b*seg, (b+1)*seg) of
-// the pass's input.  Per pass (8-bit digit at `shift`):
-//   H: block histograms of its positions -> hist[b][digit];
-//   P: one block per digit scans hist[.][digit] over the blocks ->
-//      off[b][digit] (keys of that digit in earlier blocks) and total[digit];
-//   S: block b walks its positions in tiles of 2048 in order and writes each
-//      key to  digit_base + off[b][digit] + (same digit earlier in its
-//      positions), the last term from per-warp running counts: stable.
-// The barrier's wait is bounded: past the limit the block raises
-// PLE_ERR_TIMEOUT and leaves (the result is then unspecified, nothing hangs).
+// key_hist_kernel turns the int64 rows into 32-bit keys and counts the
+// digits of every pass at once, so the global start of each digit is known
+// before the first pass.  Each pass is one sort_pass_kernel launch in which
+// a block takes one tile of kSortTile consecutive positions, in the order of
+// a ticket counter (a block only ever waits for tiles with lower tickets,
+// whose blocks are already running).  The block ranks its keys by digit
+// (warp ballots, per-warp running counts: stable) and publishes its
+// per-digit counts.  The keys of a digit in all earlier tiles are then
+// summed over three levels, so that no tile waits on a long chain:
+//   tiles of its group of 32 tiles before it (their counts);
+//   groups of its supergroup of 32 groups before its group (group totals,
+//   published by the last tile of each group);
+//   supergroups before its supergroup (totals published by the last tile of
+//   each supergroup).
+// A published word is READY | count; the count is the payload, so plain
+// relaxed loads and stores suffice.  Keys then go to digit start + earlier
+// count + rank, staged in shared memory in digit order so that the writes
+// are coalesced.  Every wait is bounded: past the limit the block raises
+// PLE_ERR_TIMEOUT and carries on with what it has (the result is then
+// unspecified; nothing hangs).
 // ---------------------------------------------------------------------------
-constexpr int kCoopThreads = 256;
-constexpr int kCoopWarps = kCoopThreads / 32;
-constexpr int kCoopItems = 4;
-constexpr int kCoopTile = kCoopThreads * kCoopItems;  // keys per tile of the scatter phase
-constexpr int kCoopMaxBlocks = 2 * kCoopThreads;      // the prefix phase scans <= 2 blocks per thread
+constexpr int kSortThreads = 256;
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kSortItems = 8;
+constexpr int kSortTile = kSortThreads * kSortItems;  // positions per tile
+constexpr int kWarpSpan = kSortTile / kSortWarps;     // positions per warp within a tile
+constexpr int kMaxPasses = 4;
+constexpr int kGroupBits = 5;                         // 32 tiles per group, 32 groups per supergroup
 constexpr unsigned kSpinLimit = 1u << 22;             // a few seconds of polling, then give up
+constexpr uint32_t kReady = 0x80000000u;              // look-back word: READY | count (count < 2^31)
 
 // Lanes of the warp holding the same BITS-bit value as this lane (valid
 // lanes only): one ballot per bit, each lane keeping the lanes that agree
@@ -76,12 +89,6 @@ __device__ __forceinline__ unsigned peers_of(bool valid, uint32_t value) {
     peers &= set ? m : ~m;
   }
   return valid ? peers : 0u;
-}
-
-// Warp-aggregated shared-memory histogram update for one key per lane.
-__device__ __forceinline__ void hist_add(uint32_t* h, bool valid, uint32_t digit) {
-  const unsigned peers = peers_of<8>(valid, digit);
-  if (valid && (peers & lanemask_lt()) == 0) atomicAdd(&h[digit], __popc(peers));
 }
 
 // Block-wide exclusive sum (every thread passes one value); *total gets the sum.
@@ -106,193 +113,245 @@ __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t x, uint32_t* wa
   return before + incl - x;
 }
 
-// Grid barrier for a cooperative grid.  The counter only grows within a call
-// (it is cleared before the launch); each arrival waits for the next multiple
-// of the grid size.
-__device__ bool grid_barrier(unsigned int* bar, unsigned int* status) {
-  __shared__ bool ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned int nblocks = gridDim.x;
-    const unsigned int old = atomicAdd(bar, 1u);
-    const unsigned int target = (old / nblocks + 1) * nblocks;
-    bool good = true;
-    for (unsigned int spins = 0;; ++spins) {
-      unsigned int v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-      if (static_cast<int>(v - target) >= 0) break;
-      if (spins >= kSpinLimit) {
-        good = false;
-        raise_flag(status, PLE_ERR_TIMEOUT);
-        break;
+__device__ __forceinline__ uint4 ld_relaxed_v4(const uint32_t* p) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ bool all_ready(const uint4& x) {
+  return (x.x & x.y & x.z & x.w & kReady) != 0;
+}
+
+// Per-digit sums of the published count rows [first, last) of one level
+// (row q: 256 words at rows + q * 256), by the whole block: warp w takes
+// rows first + w, first + w + 8, ... (up to 4 rows in flight per warp, each
+// lane reading 8 digits as two 16-byte loads); rows not yet fully published
+// are loaded again, round after round; the warps' partial sums meet in
+// `part`.  Returns the sum for digit threadIdx.x (threads < 256).
+__device__ uint32_t level_sum(const uint32_t* rows, int64_t first, int64_t last, uint32_t (*part)[kRadix],
+                              unsigned int* status) {
+  if (first >= last) return 0;  // block-uniform
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int64_t q0 = first; q0 < last; q0 += 4 * kSortWarps) {
+    uint4 x[4][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t q = q0 + warp + k * kSortWarps;
+      if (q < last) {
+        x[k][0] = ld_relaxed_v4(rows + q * kRadix + lane * 8);
+        x[k][1] = ld_relaxed_v4(rows + q * kRadix + lane * 8 + 4);
+      } else {
+        x[k][0] = x[k][1] = make_uint4(kReady, kReady, kReady, kReady);
       }
     }
-    __threadfence();
-    ok = good;
+    for (unsigned spins = 0;; ++spins) {
+      bool ready = true;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ready &= all_ready(x[k][0]) && all_ready(x[k][1]);
+      if (__all_sync(kFull, ready)) break;
+      if (spins >= kSpinLimit) {
+        if (lane == 0) raise_flag(status, PLE_ERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(64);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t q = q0 + warp + k * kSortWarps;
+        if (q < last && !(all_ready(x[k][0]) && all_ready(x[k][1]))) {
+          x[k][0] = ld_relaxed_v4(rows + q * kRadix + lane * 8);
+          x[k][1] = ld_relaxed_v4(rows + q * kRadix + lane * 8 + 4);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[0] += x[k][0].x & ~kReady; acc[1] += x[k][0].y & ~kReady;
+      acc[2] += x[k][0].z & ~kReady; acc[3] += x[k][0].w & ~kReady;
+      acc[4] += x[k][1].x & ~kReady; acc[5] += x[k][1].y & ~kReady;
+      acc[6] += x[k][1].z & ~kReady; acc[7] += x[k][1].w & ~kReady;
+    }
   }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) part[warp][lane * 8 + j] = acc[j];
   __syncthreads();
-  return ok;
+  uint32_t sum = 0;
+  if (threadIdx.x < kRadix)
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) sum += part[w][threadIdx.x];
+  __syncthreads();  // part is reused by the next level
+  return sum;
 }
 
 struct SortArgs {
-  const int64_t* rows;
   int64_t N;
-  int64_t num_rows;
+  int64_t tiles, groups, supers;
+  int passes;
   uint32_t* keys[2];
   uint32_t* vals[2];
-  uint32_t* hist[2];  // [blocks][256] per pass parity
-  uint32_t* off;    // [blocks][256]
-  uint32_t* total;  // [256]
-  unsigned int* bar;
+  uint32_t* hist;          // [kMaxPasses][256] digit totals of every pass (zeroed before the sort)
+  unsigned int* tickets;   // [kMaxPasses] tile tickets (zeroed before the sort)
+  uint32_t* look;          // [passes][tiles + groups + supers][256] published counts
   unsigned int* status;
-  unsigned int* run_done;  // [nwin] cleared here for the fold
-  int64_t nwin;
-  int passes;
 };
 
-__global__ void __launch_bounds__(kCoopThreads, 4) sort_kernel(const SortArgs a) {
-  __shared__ uint32_t h[kRadix];
-  __shared__ uint32_t wh[kCoopWarps][kRadix];
-  __shared__ uint32_t base_s[kRadix];
-  __shared__ uint32_t start_s[kRadix];
-  __shared__ uint32_t stage_k[kCoopTile];
-  __shared__ uint32_t stage_v[kCoopTile];
-  __shared__ uint32_t warp_tot[kCoopWarps];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t G = gridDim.x, b = blockIdx.x, N = a.N;
-  const int64_t seg = ((N + G - 1) / G + 31) / 32 * 32;
-  const int64_t lo = min(N, b * seg), hi = min(N, lo + seg);
-  bool bad = false;
-  for (int64_t i = b * kCoopThreads + tid; i < a.nwin; i += G * kCoopThreads) a.run_done[i] = 0;
+// Keys from the int64 rows (a row outside [0, num_rows) becomes the key
+// num_rows, sorted last and skipped by the fold) and the digit counts of
+// every pass.  Also clears the look-back words of every pass and the fold's
+// run counters.
+// Clears the digit totals and tile tickets before key_hist_kernel adds to them.
+__global__ void clear_kernel(uint32_t* words, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0;
+  allow_next_grid();
+}
 
-  // H (first pass only; later passes get their histograms from the previous
-  // scatter): histogram of this block's positions, making the keys
-  if (tid < kRadix) h[tid] = 0;
+__global__ void __launch_bounds__(kSortThreads)
+key_hist_kernel(const int64_t* __restrict__ rows, int64_t num_rows, const SortArgs a, unsigned int* run_done,
+                int64_t nwin) {
+  __shared__ uint32_t h[kMaxPasses][kRadix];
+  const int tid = threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kSortThreads;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * kSortThreads + tid;
+  for (int k = tid; k < kMaxPasses * kRadix; k += kSortThreads) (&h[0][0])[k] = 0;
+  wait_for_prior_grid();  // the totals it adds to are cleared by the previous kernel
+  const int64_t look_words = static_cast<int64_t>(a.passes) * (a.tiles + a.groups + a.supers) * kRadix;
+  for (int64_t i = g; i < look_words; i += stride) a.look[i] = 0;
+  for (int64_t i = g; i < nwin; i += stride) run_done[i] = 0;
   __syncthreads();
-  for (int64_t i0 = lo; i0 < hi; i0 += kCoopTile) {
-    uint32_t key[kCoopItems];
+  bool bad = false;
+  constexpr int kIlp = 4;  // row loads in flight per thread
+  for (int64_t i0 = g; i0 < a.N; i0 += kIlp * stride) {
+    int64_t v[kIlp];
 #pragma unroll
-    for (int r = 0; r < kCoopItems; ++r) {  // every load first
-      const int64_t i = i0 + r * kCoopThreads + tid;
-      key[r] = 0;
-      if (i < hi) {
-        const int64_t v = a.rows[i];
-        const bool ok = v >= 0 && v < a.num_rows;
+    for (int u = 0; u < kIlp; ++u) v[u] = i0 + u * stride < a.N ? __ldcs(rows + i0 + u * stride) : 0;
+#pragma unroll
+    for (int u = 0; u < kIlp; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < a.N) {
+        const bool ok = v[u] >= 0 && v[u] < num_rows;
         bad |= !ok;
-        key[r] = ok ? static_cast<uint32_t>(v) : static_cast<uint32_t>(a.num_rows);
-        a.keys[0][i] = key[r];
+        const uint32_t key = ok ? static_cast<uint32_t>(v[u]) : static_cast<uint32_t>(num_rows);
+        a.keys[0][i] = key;
+        for (int p = 0; p < a.passes; ++p) atomicAdd(&h[p][(key >> (8 * p)) & (kRadix - 1)], 1u);
       }
     }
-#pragma unroll
-    for (int r = 0; r < kCoopItems; ++r)
-      hist_add(h, i0 + r * kCoopThreads + tid < hi, key[r] & (kRadix - 1));
   }
   if (bad) raise_flag(a.status, PLE_ERR_BAD_ROW);
   __syncthreads();
-  if (tid < kRadix) a.hist[0][b * kRadix + tid] = h[tid];
-  if (!grid_barrier(a.bar, a.status)) return;
+  for (int k = tid; k < a.passes * kRadix; k += kSortThreads) {
+    const uint32_t c = (&h[0][0])[k];
+    if (c) atomicAdd(a.hist + k, c);
+  }
+  allow_next_grid();
+}
 
-  for (int p = 0; p < a.passes; ++p) {
-    const int shift = 8 * p;
-    const bool odd = p & 1, last = p + 1 == a.passes;
-    const uint32_t* kin = odd ? a.keys[1] : a.keys[0];
-    const uint32_t* vin = odd ? a.vals[1] : a.vals[0];
-    uint32_t* kout = odd ? a.keys[0] : a.keys[1];
-    uint32_t* vout = odd ? a.vals[0] : a.vals[1];
-    const uint32_t* hist = odd ? a.hist[1] : a.hist[0];
-    uint32_t* hist_next = odd ? a.hist[0] : a.hist[1];
+__global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortArgs a, const int pass) {
+  __shared__ uint32_t wh[kSortWarps][kRadix];
+  __shared__ uint32_t stage_k[kSortTile];
+  __shared__ uint32_t stage_v[kSortTile];
+  __shared__ uint32_t base_s[kRadix];
+  __shared__ uint32_t start_s[kRadix];
+  __shared__ uint32_t warp_tot[kSortWarps];
+  __shared__ int64_t tile_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  wait_for_prior_grid();
+  if (tid == 0) tile_s = atomicAdd(a.tickets + pass, 1u);
+  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
+  {  // global start of every digit of this pass (while the ticket is on its way)
+    const uint32_t c = tid < kRadix ? __ldcg(a.hist + pass * kRadix + tid) : 0;
+    uint32_t all;
+    const uint32_t start = block_exclusive_sum(c, warp_tot, &all);  // (its barriers publish tile_s and wh)
+    if (tid < kRadix) base_s[tid] = start;
+  }
+  allow_next_grid();
+  const int64_t t = tile_s;
+  const int64_t N = a.N, i0 = t * kSortTile + warp * kWarpSpan;
+  const int shift = 8 * pass;
+  const bool odd = pass & 1;  // (selects, not indexes: the parameter arrays stay in the constant bank)
+  const uint32_t* kin = odd ? a.keys[1] : a.keys[0];
+  const uint32_t* vin = odd ? a.vals[1] : a.vals[0];
+  uint32_t* kout = odd ? a.keys[0] : a.keys[1];
+  uint32_t* vout = odd ? a.vals[0] : a.vals[1];
 
-    // P: per digit, exclusive scan over the blocks (two blocks per thread);
-    // every block also clears its row of the next pass's histogram
-    for (int d = static_cast<int>(b); d < kRadix; d += static_cast<int>(G)) {
-      const int64_t b0 = 2 * tid, b1 = 2 * tid + 1;
-      const uint32_t v0 = b0 < G ? __ldcg(hist + b0 * kRadix + d) : 0;
-      const uint32_t v1 = b1 < G ? __ldcg(hist + b1 * kRadix + d) : 0;
-      uint32_t tot;
-      const uint32_t ex = block_exclusive_sum(v0 + v1, warp_tot, &tot);
-      if (b0 < G) a.off[b0 * kRadix + d] = ex;
-      if (b1 < G) a.off[b1 * kRadix + d] = ex + v0;
-      if (tid == 0) a.total[d] = tot;
+  uint32_t key[kSortItems], val[kSortItems];
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r) {
+    const int64_t i = i0 + r * 32 + lane;
+    key[r] = i < N ? kin[i] : 0;
+    val[r] = i < N ? (pass == 0 ? static_cast<uint32_t>(i) : vin[i]) : 0;
+  }
+  // rank among the same digit within the warp's positions, in order
+  uint8_t rank[kSortItems];
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r) {
+    const bool valid = i0 + r * 32 + lane < N;
+    const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
+    const unsigned peers = peers_of<8>(valid, digit);
+    const unsigned lower = __popc(peers & lanemask_lt());
+    rank[r] = valid ? static_cast<uint8_t>(wh[warp][digit] + lower) : 0;  // < 256 keys per warp
+    __syncwarp();
+    if (valid && lower == 0) wh[warp][digit] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  uint32_t count = 0;  // keys of digit tid in this tile; wh becomes the per-warp offsets
+  if (tid < kRadix) {
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = wh[w][tid];
+      wh[w][tid] = count;
+      count += c;
     }
-    if (!last && tid < kRadix) hist_next[b * kRadix + tid] = 0;
-    if (!grid_barrier(a.bar, a.status)) return;
-
-    // S: stable scatter of this block's positions, tile by tile
-    uint32_t key[kCoopItems], val[kCoopItems];
-    auto load_tile = [&](int64_t i0) {
+  }
+  if (tid < kRadix)  // this tile's counts, as early as possible
+    st_relaxed(a.look + (static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) + t) * kRadix + tid,
+               kReady | count);
+  // stage the tile in digit order (tile-local positions need no other tile)
+  uint32_t tile_n;
+  const uint32_t local_start = block_exclusive_sum(tid < kRadix ? count : 0u, warp_tot, &tile_n);
+  if (tid < kRadix) start_s[tid] = local_start;
+  __syncthreads();
 #pragma unroll
-      for (int r = 0; r < kCoopItems; ++r) {
-        const int64_t i = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane;
-        key[r] = i < hi ? kin[i] : 0;
-        val[r] = i < hi ? (p == 0 ? static_cast<uint32_t>(i) : vin[i]) : 0;
-      }
-    };
-    if (lo < hi) load_tile(lo);  // in flight during the digit-base scan
-    {
-      const uint32_t t = tid < kRadix ? __ldcg(a.total + tid) : 0;
-      const uint32_t mine = tid < kRadix ? __ldcg(a.off + b * kRadix + tid) : 0;
-      uint32_t all;
-      const uint32_t digit_base = block_exclusive_sum(t, warp_tot, &all);
-      if (tid < kRadix) base_s[tid] = digit_base + mine;
+  for (int r = 0; r < kSortItems; ++r) {
+    if (i0 + r * 32 + lane < N) {
+      const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
+      const uint32_t pos = start_s[digit] + wh[warp][digit] + rank[r];
+      stage_k[pos] = key[r];
+      stage_v[pos] = val[r];
     }
-    for (int64_t i0 = lo; i0 < hi; i0 += kCoopTile) {
-      for (int k = tid; k < kCoopWarps * kRadix; k += kCoopThreads) (&wh[0][0])[k] = 0;
-      __syncthreads();
-      uint8_t rank[kCoopItems];
-#pragma unroll
-      for (int r = 0; r < kCoopItems; ++r) {
-        const bool valid = i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi;
-        const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-        const unsigned peers = peers_of<8>(valid, digit);
-        const unsigned lower = __popc(peers & lanemask_lt());
-        rank[r] = valid ? static_cast<uint8_t>(wh[warp][digit] + lower) : 0;
-        __syncwarp();
-        if (valid && lower == 0) wh[warp][digit] += __popc(peers);
-        __syncwarp();
-      }
-      __syncthreads();
-      uint32_t tile_count = 0;
-      if (tid < kRadix) {
-#pragma unroll
-        for (int w = 0; w < kCoopWarps; ++w) {
-          const uint32_t c = wh[w][tid];
-          wh[w][tid] = tile_count;
-          tile_count += c;
-        }
-      }
-      // tile-local start of every digit, then stage the tile in digit order
-      uint32_t tile_n;
-      const uint32_t local_start = block_exclusive_sum(tid < kRadix ? tile_count : 0u, warp_tot, &tile_n);
-      if (tid < kRadix) start_s[tid] = local_start;
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < kCoopItems; ++r) {
-        if (i0 + warp * (kCoopTile / kCoopWarps) + r * 32 + lane < hi) {
-          const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-          const uint32_t pos = start_s[digit] + wh[warp][digit] + rank[r];
-          stage_k[pos] = key[r];
-          stage_v[pos] = val[r];
-        }
-      }
-      __syncthreads();
-      // coalesced writes: consecutive threads, consecutive destinations within a digit
-      for (uint32_t j = tid; j < tile_n; j += kCoopThreads) {
-        const uint32_t k2 = stage_k[j];
-        const uint32_t digit = (k2 >> shift) & (kRadix - 1);
-        const uint32_t dst = base_s[digit] + (j - start_s[digit]);
-        if (dst < N) {  // always true when the counts are consistent
-          kout[dst] = k2;
-          vout[dst] = stage_v[j];
-          if (!last)  // histogram of the next pass, by destination block
-            atomicAdd(hist_next + static_cast<uint32_t>(dst / seg) * kRadix + ((k2 >> (shift + 8)) & (kRadix - 1)), 1u);
-        }
-      }
-      __syncthreads();
-      if (tid < kRadix) base_s[tid] += tile_count;
-      if (i0 + kCoopTile < hi) load_tile(i0 + kCoopTile);
+  }
+  __syncthreads();  // the staging's reads of wh are done: it holds the look-back's partial sums now
+  // keys of digit tid in the earlier tiles, over the three levels
+  {
+    const uint32_t* tile_rows = a.look + static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) * kRadix;
+    uint32_t* group_rows = const_cast<uint32_t*>(tile_rows) + a.tiles * kRadix;
+    uint32_t* super_rows = group_rows + a.groups * kRadix;
+    const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
+    uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
+    if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
+    before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
+    if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
+    before += level_sum(super_rows, 0, sg, wh, a.status);
+    if (tid < kRadix) base_s[tid] += before;
+  }
+  __syncthreads();
+  // coalesced writes: consecutive threads, consecutive destinations within a digit
+  for (uint32_t j = tid; j < tile_n; j += kSortThreads) {
+    const uint32_t k2 = stage_k[j];
+    const uint32_t digit = (k2 >> shift) & (kRadix - 1);
+    const uint32_t dst = base_s[digit] + (j - start_s[digit]);
+    if (dst < N) {  // always true when the counts are consistent
+      kout[dst] = k2;
+      vout[dst] = stage_v[j];
     }
-    if (!last && !grid_barrier(a.bar, a.status)) return;
   }
 }
 
@@ -832,9 +891,9 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
 // host side
 // ---------------------------------------------------------------------------
 struct Layout {
-  size_t keys[2], vals[2], hist[2], off, total, csum, run_len, run_done, zeroed, total_bytes;
-  size_t zeroed_bytes;  // the sort's barrier counter (and a spare word), cleared per call
-  int64_t nwin;
+  size_t keys[2], vals[2], look, csum, run_len, run_done, zeroed, total_bytes;
+  size_t zeroed_bytes;  // digit totals of every pass and the tile tickets, cleared per call
+  int64_t nwin, tiles, groups, supers;
 };
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t{255}; }
@@ -842,6 +901,9 @@ size_t align_up(size_t x) { return (x + 255) & ~size_t{255}; }
 Layout layout_for(int64_t N, int D) {
   Layout L{};
   L.nwin = (N + 31) / 32;
+  L.tiles = (N + kSortTile - 1) / kSortTile;
+  L.groups = (L.tiles + 31) >> kGroupBits;
+  L.supers = (L.groups + 31) >> kGroupBits;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -850,35 +912,14 @@ Layout layout_for(int64_t N, int D) {
   };
   for (int b = 0; b < 2; ++b) L.keys[b] = take(sizeof(uint32_t) * N);
   for (int b = 0; b < 2; ++b) L.vals[b] = take(sizeof(uint32_t) * N);
-  L.hist[0] = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
-  L.hist[1] = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
-  L.off = take(sizeof(uint32_t) * kRadix * kCoopMaxBlocks);
-  L.total = take(sizeof(uint32_t) * kRadix);
+  L.look = take(sizeof(uint32_t) * kRadix * kMaxPasses * static_cast<size_t>(L.tiles + L.groups + L.supers));
   L.csum = take(sizeof(float) * 2 * static_cast<size_t>(L.nwin) * D);
   L.run_len = take(sizeof(int) * L.nwin);
   L.run_done = take(sizeof(unsigned int) * L.nwin);
-  L.zeroed_bytes = 2 * sizeof(unsigned int);
+  L.zeroed_bytes = sizeof(uint32_t) * (kMaxPasses * kRadix + kMaxPasses);
   L.zeroed = take(L.zeroed_bytes);
   L.total_bytes = off;
   return L;
-}
-
-// Blocks of the cooperative sort: all resident at once, at most one tile each
-// when the input is small.
-int sort_blocks(int64_t N, cudaError_t* err) {
-  static std::atomic<int> per_sm_cache[64];
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return 0;
-  int per_sm = (dev >= 0 && dev < 64) ? per_sm_cache[dev].load(std::memory_order_relaxed) : 0;
-  if (per_sm <= 0) {
-    *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sort_kernel, kCoopThreads, 0);
-    if (*err != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) per_sm_cache[dev].store(per_sm, std::memory_order_relaxed);
-  }
-  const int64_t resident = static_cast<int64_t>(per_sm) * sm_count();
-  const int64_t tiles = (N + kCoopTile - 1) / kCoopTile;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({resident, tiles, int64_t{kCoopMaxBlocks}})));
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -929,39 +970,41 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   auto* ws = static_cast<unsigned char*>(workspace);
   const auto s = static_cast<cudaStream_t>(stream);
   SortArgs sa{};
-  sa.rows = rows;
   sa.N = N;
-  sa.num_rows = plan->num_rows;
+  sa.tiles = L.tiles;
+  sa.groups = L.groups;
+  sa.supers = L.supers;
   for (int b = 0; b < 2; ++b) {
     sa.keys[b] = reinterpret_cast<uint32_t*>(ws + L.keys[b]);
     sa.vals[b] = reinterpret_cast<uint32_t*>(ws + L.vals[b]);
   }
-  sa.hist[0] = reinterpret_cast<uint32_t*>(ws + L.hist[0]);
-  sa.hist[1] = reinterpret_cast<uint32_t*>(ws + L.hist[1]);
-  sa.off = reinterpret_cast<uint32_t*>(ws + L.off);
-  sa.total = reinterpret_cast<uint32_t*>(ws + L.total);
-  sa.bar = reinterpret_cast<unsigned int*>(ws + L.zeroed);
+  sa.look = reinterpret_cast<uint32_t*>(ws + L.look);
+  sa.hist = reinterpret_cast<uint32_t*>(ws + L.zeroed);
+  sa.tickets = sa.hist + kMaxPasses * kRadix;
   sa.status = status;
   float* csum = reinterpret_cast<float*>(ws + L.csum);
   RunBook rb;
   rb.len = reinterpret_cast<int*>(ws + L.run_len);
   rb.done = reinterpret_cast<unsigned int*>(ws + L.run_done);
-  sa.run_done = rb.done;
-  sa.nwin = L.nwin;
 
   // key bits: keys lie in [0, num_rows] (num_rows marks a bad row)
   int bits = 0;
   while (bits < 32 && (static_cast<uint64_t>(plan->num_rows) >> bits) != 0) ++bits;
   sa.passes = std::max(1, (bits + 7) / 8);
 
-  e = cudaMemsetAsync(sa.bar, 0, L.zeroed_bytes, s);
+  clear_kernel<<<1, kSortThreads, 0, s>>>(reinterpret_cast<uint32_t*>(ws + L.zeroed),
+                                          static_cast<int>(L.zeroed_bytes / sizeof(uint32_t)));
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
-  const int blocks = sort_blocks(N, &e);
-  if (blocks <= 0) return cuda_fail(e);
-  void* kargs[] = {&sa};
-  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(sort_kernel), dim3(blocks), dim3(kCoopThreads),
-                                  kargs, 0, s);
+  // few blocks: each adds its digit counts to the same 256 * passes totals
+  const int64_t hist_blocks = std::min<int64_t>((N + kSortThreads - 1) / kSortThreads, int64_t{2} * sm_count());
+  e = launch_after(key_hist_kernel, dim3(static_cast<unsigned>(hist_blocks)), dim3(kSortThreads), 0, s, rows,
+                   plan->num_rows, sa, rb.done, L.nwin);
   if (e != cudaSuccess) return cuda_fail(e);
+  for (int p = 0; p < sa.passes; ++p) {
+    e = launch_after(sort_pass_kernel, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s, sa, p);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   const uint32_t* Ks = sa.keys[sa.passes & 1];
   const uint32_t* Is = sa.vals[sa.passes & 1];
   const uint32_t bad_key = static_cast<uint32_t>(plan->num_rows);
@@ -985,7 +1028,6 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
              : fold(fold_generic_kernel<false>, fold_grid, kFoldThreads, 0);
   }
 #undef PLE_WIDE
-  if (e != cudaSuccess) return cuda_fail(e);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }
