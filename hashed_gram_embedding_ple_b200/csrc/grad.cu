@@ -617,16 +617,6 @@ __device__ __forceinline__ void red_add4(float* p, float a, float b, float c, fl
   asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
-template <bool BF16>
-__device__ __forceinline__ void unpack16(const uint4& y, float* v) {
-  if constexpr (BF16) {
-    v[0] = bf16_lo(y.x); v[1] = bf16_hi(y.x); v[2] = bf16_lo(y.y); v[3] = bf16_hi(y.y);
-    v[4] = bf16_lo(y.z); v[5] = bf16_hi(y.z); v[6] = bf16_lo(y.w); v[7] = bf16_hi(y.w);
-  } else {
-    v[0] = __uint_as_float(y.x); v[1] = __uint_as_float(y.y);
-    v[2] = __uint_as_float(y.z); v[3] = __uint_as_float(y.w);
-  }
-}
 
 // Second level of a long run, by a whole warp after its window is folded:
 // the run's chunk sums go through the warp's staging buffer (`stage_vecs`
@@ -673,18 +663,47 @@ __device__ void finish_run_staged(const float* csum, int64_t s, int nc, int D, u
 // taken in rounds of whole chunks covering at most kWideRows positions (a
 // chunk has at most 32 hits, so it never straddles two rounds); the rows of
 // a round are staged in shared memory with asynchronous copies in one round
-// trip.  The L-lane groups of the warp then take the round's chunks in turn
-// (chunk k to group k mod 32/L) and fold them independently from shared
-// memory, each in the fixed order, lane `sub` of a group owning CPLN =
-// 16/elem columns.  A finished chunk that is a whole run is added into
+// trip.  The L-lane groups of the warp then fold the round's chunks
+// independently from shared memory, each in the fixed order, lane `sub` of a
+// group owning CPLN = 16/elem columns; group g takes the chunks that start at
+// a position = g modulo the number of groups (32/L), so it only visits its
+// own chunks.  A finished chunk that is a whole run is added into
 // table_grad by its group; otherwise it goes to its chunk-sum slot.
 constexpr int kWideRows = 32;  // staged rows per warp and round
+
+// Columns of the staged grad row that lane `sub` of an L-lane group folds:
+// 4-column blocks at 4*sub + 4*L*h, h = 0 .. CPLN/4 - 1 (fp32 grad: one block,
+// the lane's own 16 bytes; bf16 grad: two blocks, one from each half of the
+// row).  So every 16-byte fp32 reduction instruction of the group covers 4*L
+// consecutive columns of the table_grad row: whole sectors.
+template <int L, bool BF16>
+__device__ __forceinline__ int lane_col(int sub, int q) {  // fp32 column of acc[q], q a multiple of 4
+  return 4 * sub + L * q;
+}
+
+template <int L, bool BF16>
+__device__ __forceinline__ void load_lane_cols(const uint4* row, int sub, float* v) {
+  if constexpr (BF16) {
+    const uint2* r = reinterpret_cast<const uint2*>(row);  // 4 bf16 per 8 bytes
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint2 y = r[sub + L * h];
+      v[4 * h] = bf16_lo(y.x); v[4 * h + 1] = bf16_hi(y.x); v[4 * h + 2] = bf16_lo(y.y); v[4 * h + 3] = bf16_hi(y.y);
+    }
+  } else {
+    const uint4 y = row[sub];
+    v[0] = __uint_as_float(y.x); v[1] = __uint_as_float(y.y); v[2] = __uint_as_float(y.z); v[3] = __uint_as_float(y.w);
+  }
+}
 
 template <int L>
 __host__ __device__ constexpr int wide_warps() {
   return L >= 32 ? 2 : L >= 16 ? 4 : 8;  // about 33 KB of staging per block
 }
-constexpr int kWideTail = 64 * 4 + 48;  // per warp after the rows: 64 keys, 2 pending long runs, a count
+// per warp after the rows: 64 keys, 64 hit ids, 32 chunk descriptors, 2 pending long runs, a count
+constexpr int kWideTail = 64 * 4 + 64 * 4 + 32 * 4 + 48;
+constexpr uint32_t kChunkWhole = 1u << 8;  // chunk descriptor: the chunk is a whole run
+constexpr uint32_t kChunkSkip = 1u << 9;   // chunk descriptor: rows outside the table (dropped)
 
 template <int L>
 __host__ __device__ constexpr size_t wide_smem() {
@@ -696,6 +715,14 @@ struct PendingRun {
   int nc;
   uint32_t key;
 };
+
+// Bits 0, n, 2n, ... of a 64-bit word.
+template <int n>
+__host__ __device__ constexpr uint64_t every_nth_bit() {
+  uint64_t m = 0;
+  for (int b = 0; b < 64; b += n) m |= 1ull << b;
+  return m;
+}
 
 template <int L>
 __host__ __device__ constexpr int wide_min_blocks() {
@@ -714,7 +741,9 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   const int grp = lane / L, sub = lane % L;
   uint4* rows_s = reinterpret_cast<uint4*>(wide_smem_raw + warp * (kWideRows * L * 16 + kWideTail));
   uint32_t* keys_s = reinterpret_cast<uint32_t*>(rows_s + kWideRows * L);  // 64 keys
-  PendingRun* pend = reinterpret_cast<PendingRun*>(keys_s + 64);           // long runs this warp completed
+  uint32_t* ids_s = keys_s + 64;                                           // 64 hit ids
+  uint32_t* desc_s = ids_s + 64;                                           // 32 chunk descriptors
+  PendingRun* pend = reinterpret_cast<PendingRun*>(desc_s + 32);           // long runs this warp completed
   int* npend = reinterpret_cast<int*>(pend + 2);
   const int64_t w = static_cast<int64_t>(blockIdx.x) * wide_warps<L>() + warp;
   wait_for_prior_grid();
@@ -726,12 +755,13 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
   keys_s[lane] = W.kA;
   keys_s[32 + lane] = W.kB;
+  ids_s[lane] = W.iA;
+  ids_s[32 + lane] = W.iB;
   if (lane == 0) *npend = 0;
   __syncwarp();
 
   const uint64_t in_range = (W.b >= 64 ? ~0ull : ((1ull << W.b) - 1)) & ~((1ull << W.a) - 1);
   uint64_t rem = W.cm & in_range;  // chunk starts still to fold
-  int k = 0;
   while (rem) {
     // the round: whole chunks from the first remaining start, at most kWideRows positions
     const int r0 = __ffsll(static_cast<long long>(rem)) - 1;
@@ -740,41 +770,61 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
       const uint64_t later = rem & ~(1ull << r0) & ((2ull << (r0 + kWideRows)) - 1);
       r1 = 63 - __clzll(later);  // a later chunk start within reach exists: chunks are <= 32 long
     }
-    for (int i0 = 0; i0 < r1 - r0; i0 += RPI) {  // uniform trip count: the shuffles see every lane
-      const int e = r0 + i0 + grp;
-      const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
-      if (e < r1)
-        cp_async16(rows_s + (e - r0) * L + sub, gbase + static_cast<size_t>(e < 32 ? ia : ib) * row_bytes);
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    __syncwarp();
-    uint64_t starts = rem & ((r1 >= 64 ? ~0ull : ((1ull << r1) - 1)));
+    for (int e = r0 + grp; e < r1; e += RPI)
+      cp_async16(rows_s + (e - r0) * L + sub, gbase + static_cast<size_t>(ids_s[e]) * row_bytes);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const uint64_t starts = rem & ((r1 >= 64 ? ~0ull : ((1ull << r1) - 1)));
     rem &= ~starts;
-    while (starts) {
-      const int c = __ffsll(static_cast<long long>(starts)) - 1;
-      starts &= starts - 1;
-      if ((k++ % RPI) != grp) continue;  // another group's chunk
-      const int nxt = starts ? __ffsll(static_cast<long long>(starts)) - 1 : r1;
+    // chunk starts of the round relative to r0 (a round spans at most 32 positions); lane j
+    // describes the chunk starting at r0 + j (while the rows are on their way): where it ends,
+    // whether it is a whole run, whether its rows are outside the table
+    const uint32_t st32 = static_cast<uint32_t>(starts >> r0);
+    if ((st32 >> lane) & 1u) {
+      const uint32_t above = st32 & ~((2u << lane) - 1u);  // (lane 31: 2u << 31 wraps to 0, nothing above)
+      const int nrel = above ? __ffs(above) - 1 : r1 - r0;
+      const int c = r0 + lane, nxt = r0 + nrel;
+      const bool is_head = (W.hm >> c) & 1ull;
+      const bool run_ends = (W.p0 + nxt >= N) || ((W.hm >> nxt) & 1ull);  // nxt < 64 unless the data ends there
+      desc_s[lane] = static_cast<uint32_t>(nrel) | (is_head && run_ends ? kChunkWhole : 0u) |
+                     (keys_s[c] == bad_key ? kChunkSkip : 0u);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    // this group's chunks: those starting at a position = grp mod RPI (relative position
+    // j = c - r0, so j = grp - r0 mod RPI)
+    uint32_t mine = st32 & static_cast<uint32_t>(every_nth_bit<RPI>() >> ((r0 - grp) & (RPI - 1)));
+    while (mine) {
+      const int j = __ffs(mine) - 1;
+      mine &= mine - 1;
+      const uint32_t dsc = desc_s[j];
+      if (dsc & kChunkSkip) continue;
+      const int nrel = static_cast<int>(dsc & 0xFFu);
       float acc[CPLN];
-      unpack16<BF16>(rows_s[(c - r0) * L + sub], acc);
-      for (int e = c + 1; e < nxt; ++e) {
+      load_lane_cols<L, BF16>(rows_s + j * L, sub, acc);
+      for (int e = j + 1; e < nrel; ++e) {
         float v[CPLN];
-        unpack16<BF16>(rows_s[(e - r0) * L + sub], v);
+        load_lane_cols<L, BF16>(rows_s + e * L, sub, v);
 #pragma unroll
         for (int q = 0; q < CPLN; ++q) acc[q] = acc[q] + v[q];
       }
+      const int c = r0 + j;
       const uint32_t key = keys_s[c];
-      if (key == bad_key) continue;
-      int64_t slot = 0;
-      if (chunk_is_whole_run(W, c, nxt, N, &slot)) {
-        float* dst = table_grad + static_cast<int64_t>(key) * D + sub * CPLN;
+      if (dsc & kChunkWhole) {
+        float* dst = table_grad + static_cast<int64_t>(key) * D;
 #pragma unroll
-        for (int q = 0; q < CPLN; q += 4) red_add4(dst + q, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+        for (int q = 0; q < CPLN; q += 4) {
+          float* d4 = dst + lane_col<L, BF16>(sub, q);
+          red_add4(d4, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+        }
       } else {
-        float* dst = csum + slot * D + sub * CPLN;
+        const int nxt = r0 + nrel;
+        const bool is_head = (W.hm >> c) & 1ull;
+        const int64_t slot = 2 * ((W.p0 + c) >> 5) + (is_head ? 1 : 0);
+        float* dst = csum + slot * D;
 #pragma unroll
         for (int q = 0; q < CPLN; q += 4)
-          *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+          *reinterpret_cast<float4*>(dst + lane_col<L, BF16>(sub, q)) =
+              make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
         const unsigned gmask = L == 32 ? kFull : (((1u << L) - 1u) << (grp * L));
         int64_t s = 0;
         const int nc = chunk_stored(W, c, nxt, N, gmask, grp * L, rb, &s);
@@ -784,7 +834,7 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
         }
       }
     }
-    __syncwarp();  // the next round reuses the staging buffer
+    __syncwarp();  // the next round reuses the staging buffer and the descriptors
   }
   const int n = min(*npend, 2);
   for (int q = 0; q < n; ++q)
