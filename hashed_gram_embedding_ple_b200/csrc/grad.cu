@@ -209,6 +209,7 @@ struct SortArgs {
 // run counters.
 // Clears the digit totals and tile tickets before key_hist_kernel adds to them.
 __global__ void clear_kernel(uint32_t* words, int n) {
+  wait_for_prior_grid();  // (launched early, behind the caller's previous kernel)
   for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0;
   allow_next_grid();
 }
@@ -264,11 +265,11 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   wait_for_prior_grid();
   if (tid == 0) tile_s = atomicAdd(a.tickets + pass, 1u);
-  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
+  if (tid < kRadix) start_s[tid] = 0;  // the tile's digit counts first
   {  // global start of every digit of this pass (while the ticket is on its way)
     const uint32_t c = tid < kRadix ? __ldcg(a.hist + pass * kRadix + tid) : 0;
     uint32_t all;
-    const uint32_t start = block_exclusive_sum(c, warp_tot, &all);  // (its barriers publish tile_s and wh)
+    const uint32_t start = block_exclusive_sum(c, warp_tot, &all);  // (its barriers publish tile_s, start_s)
     if (tid < kRadix) base_s[tid] = start;
   }
   allow_next_grid();
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
   const uint32_t* vin = odd ? a.vals[1] : a.vals[0];
   uint32_t* kout = odd ? a.keys[0] : a.keys[1];
   uint32_t* vout = odd ? a.vals[0] : a.vals[1];
+  uint32_t* tile_rows = a.look + static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) * kRadix;
 
   uint32_t key[kSortItems], val[kSortItems];
 #pragma unroll
@@ -288,6 +290,32 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
     key[r] = i < N ? kin[i] : 0;
     val[r] = i < N ? (pass == 0 ? static_cast<uint32_t>(i) : vin[i]) : 0;
   }
+  // digit counts of the tile (shared-memory atomics), published at once so
+  // that later tiles' look-backs do not wait for this tile's ranking
+#pragma unroll
+  for (int r = 0; r < kSortItems; ++r)
+    if (i0 + r * 32 + lane < N) atomicAdd(&start_s[(key[r] >> shift) & (kRadix - 1)], 1u);
+  __syncthreads();
+  const uint32_t count = tid < kRadix ? start_s[tid] : 0;  // keys of digit tid in this tile
+  if (tid < kRadix) st_relaxed(tile_rows + t * kRadix + tid, kReady | count);
+  // keys of digit tid in the earlier tiles, over the three levels (wh is the scratch)
+  {
+    uint32_t* group_rows = tile_rows + a.tiles * kRadix;
+    uint32_t* super_rows = group_rows + a.groups * kRadix;
+    const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
+    uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
+    if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
+    before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
+    if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
+    before += level_sum(super_rows, 0, sg, wh, a.status);
+    if (tid < kRadix) base_s[tid] += before;
+  }
+  // tile-local start of every digit
+  uint32_t tile_n;
+  const uint32_t local_start = block_exclusive_sum(count, warp_tot, &tile_n);
+  if (tid < kRadix) start_s[tid] = local_start;
+  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
+  __syncthreads();
   // rank among the same digit within the warp's positions, in order
   uint8_t rank[kSortItems];
 #pragma unroll
@@ -302,23 +330,18 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
     __syncwarp();
   }
   __syncthreads();
-  uint32_t count = 0;  // keys of digit tid in this tile; wh becomes the per-warp offsets
-  if (tid < kRadix) {
+  if (tid < kRadix) {  // per-warp offsets within each digit
+    uint32_t run = 0;
 #pragma unroll
     for (int w = 0; w < kSortWarps; ++w) {
       const uint32_t c = wh[w][tid];
-      wh[w][tid] = count;
-      count += c;
+      wh[w][tid] = run;
+      run += c;
     }
   }
-  if (tid < kRadix)  // this tile's counts, as early as possible
-    st_relaxed(a.look + (static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) + t) * kRadix + tid,
-               kReady | count);
-  // stage the tile in digit order (tile-local positions need no other tile)
-  uint32_t tile_n;
-  const uint32_t local_start = block_exclusive_sum(tid < kRadix ? count : 0u, warp_tot, &tile_n);
-  if (tid < kRadix) start_s[tid] = local_start;
   __syncthreads();
+  // stage the tile in digit order, then coalesced writes: consecutive
+  // threads, consecutive destinations within a digit
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
     if (i0 + r * 32 + lane < N) {
@@ -328,22 +351,7 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
       stage_v[pos] = val[r];
     }
   }
-  __syncthreads();  // the staging's reads of wh are done: it holds the look-back's partial sums now
-  // keys of digit tid in the earlier tiles, over the three levels
-  {
-    const uint32_t* tile_rows = a.look + static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) * kRadix;
-    uint32_t* group_rows = const_cast<uint32_t*>(tile_rows) + a.tiles * kRadix;
-    uint32_t* super_rows = group_rows + a.groups * kRadix;
-    const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
-    uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
-    if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
-    before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
-    if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
-    before += level_sum(super_rows, 0, sg, wh, a.status);
-    if (tid < kRadix) base_s[tid] += before;
-  }
   __syncthreads();
-  // coalesced writes: consecutive threads, consecutive destinations within a digit
   for (uint32_t j = tid; j < tile_n; j += kSortThreads) {
     const uint32_t k2 = stage_k[j];
     const uint32_t digit = (k2 >> shift) & (kRadix - 1);
@@ -1042,9 +1050,8 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
   while (bits < 32 && (static_cast<uint64_t>(plan->num_rows) >> bits) != 0) ++bits;
   sa.passes = std::max(1, (bits + 7) / 8);
 
-  clear_kernel<<<1, kSortThreads, 0, s>>>(reinterpret_cast<uint32_t*>(ws + L.zeroed),
-                                          static_cast<int>(L.zeroed_bytes / sizeof(uint32_t)));
-  e = cudaGetLastError();
+  e = launch_after(clear_kernel, dim3(1), dim3(kSortThreads), 0, s, reinterpret_cast<uint32_t*>(ws + L.zeroed),
+                   static_cast<int>(L.zeroed_bytes / sizeof(uint32_t)));
   if (e != cudaSuccess) return cuda_fail(e);
   // few blocks: each adds its digit counts to the same 256 * passes totals
   const int64_t hist_blocks = std::min<int64_t>((N + kSortThreads - 1) / kSortThreads, int64_t{2} * sm_count());

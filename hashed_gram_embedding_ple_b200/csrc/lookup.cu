@@ -281,6 +281,7 @@ lookup_kernel(const HashParams hp, const int64_t* __restrict__ tokens, int64_t T
   load_consts(hp, consts);
   check_seqlens(cu, num_seqs, T, status);
   __syncthreads();
+  allow_next_grid();  // a dependent launch waits for this grid's completion before it reads anything
 
   const int64_t Tout = kSlice ? om.count : T;
   const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + warp) * TW;  // first output token
