@@ -69,6 +69,14 @@ def _load():
         lib.oracle_ple_grad_apply.argtypes = [_i64p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int,
                                               ctypes.c_int32, ctypes.c_int64, _f32p]
         lib.oracle_ple_grad_apply.restype = ctypes.c_int
+        _f64p = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_conv_forward.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int32, _f64p,
+                                            ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, _f64p]
+        lib.oracle_conv_forward.restype = ctypes.c_int
+        lib.oracle_conv_backward.argtypes = [_f64p, _f64p, ctypes.c_int64, ctypes.c_int64, _i32p, ctypes.c_int32,
+                                             _f64p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_conv_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -189,3 +197,46 @@ def grad_apply(rows_, grad, table_grad: np.ndarray) -> np.ndarray:
     if rc != 0:
         raise ValueError("row outside the table")
     return table_grad
+
+
+# ---------------------------------------------------------------------------
+# segment-aware causal dilated depthwise convolution (PLE layer's short conv)
+# ---------------------------------------------------------------------------
+_f64p = ctypes.POINTER(ctypes.c_double)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def conv_forward(x, cu_seqlens, w, dilation: int, bias=None) -> np.ndarray:
+    """y [T, C] of the segment-aware causal dilated depthwise convolution of x [T, C]
+    with filters w [C, K] (tap k reads dilation*(K-1-k) tokens back, zero before the
+    segment start) plus bias [C]; fp64."""
+    x, w = _f64(x), _f64(w)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T, C = x.shape
+    K = w.shape[1]
+    b = None if bias is None else _f64(bias)
+    y = np.empty((T, C), np.float64)
+    rc = _load().oracle_conv_forward(_p(x, _f64p), T, C, _p(cu, _i32p), len(cu) - 1, _p(w, _f64p), K, int(dilation),
+                                     None if b is None else b.ctypes.data, _p(y, _f64p))
+    if rc != 0:
+        raise ValueError(f"bad conv arguments ({rc})")
+    return y
+
+
+def conv_backward(dy, x, cu_seqlens, w, dilation: int):
+    """(dx [T, C], dw [C, K], db [C]) of conv_forward for the output gradient dy; fp64."""
+    dy, x, w = _f64(dy), _f64(x), _f64(w)
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    T, C = x.shape
+    K = w.shape[1]
+    dx = np.empty((T, C), np.float64)
+    dw = np.empty((C, K), np.float64)
+    db = np.empty(C, np.float64)
+    rc = _load().oracle_conv_backward(_p(dy, _f64p), _p(x, _f64p), T, C, _p(cu, _i32p), len(cu) - 1, _p(w, _f64p),
+                                      K, int(dilation), dx.ctypes.data, dw.ctypes.data, db.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"bad conv arguments ({rc})")
+    return dx, dw, db

@@ -279,4 +279,63 @@ int oracle_ple_grad_apply(const int64_t* rows, int64_t N, const void* grad, int 
   return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Segment-aware causal dilated depthwise convolution (NeMo AutoModel engram
+// API page, Qwen3_8_FlashNextPLELayer._causal_short_conv and
+// _segmented_conv): every packed segment is convolved as if it started a
+// fresh row, with (K-1)*dilation zeros of history ahead of it, one filter of
+// K taps per channel (depthwise), tap k reading the position
+// dilation*(K-1-k) tokens back.  Plain fp64 loops in the order of that
+// definition.
+// ---------------------------------------------------------------------------
+int oracle_conv_forward(const double* x, int64_t T, int64_t C, const int32_t* cu_seqlens, int32_t num_seqs,
+                        const double* w, int32_t K, int32_t dilation, const double* bias, double* y) {
+  if (T < 0 || C < 1 || K < 1 || dilation < 1 || num_seqs < 1) return -1;
+  if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T) return -2;
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int64_t start = cu_seqlens[s];
+    for (int64_t t = start; t < cu_seqlens[s + 1]; ++t) {
+      for (int64_t c = 0; c < C; ++c) {
+        double acc = bias != nullptr ? bias[c] : 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+          const int64_t src = t - static_cast<int64_t>(dilation) * (K - 1 - k);
+          if (src >= start) acc += w[c * K + k] * x[src * C + c];  // before the segment: zero history
+        }
+        y[t * C + c] = acc;
+      }
+    }
+  }
+  return 0;
+}
+
+// Gradients of the convolution above for an output gradient dy: every tap
+// (t, k) that read x[src, c] sends w[c, k] * dy[t, c] to dx[src, c] and
+// dy[t, c] * x[src, c] to dw[c, k]; db[c] sums dy[., c].  dx, dw and db are
+// overwritten; any of them may be null.
+int oracle_conv_backward(const double* dy, const double* x, int64_t T, int64_t C, const int32_t* cu_seqlens,
+                         int32_t num_seqs, const double* w, int32_t K, int32_t dilation, double* dx, double* dw,
+                         double* db) {
+  if (T < 0 || C < 1 || K < 1 || dilation < 1 || num_seqs < 1) return -1;
+  if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T) return -2;
+  if (dx != nullptr) std::fill(dx, dx + T * C, 0.0);
+  if (dw != nullptr) std::fill(dw, dw + C * K, 0.0);
+  if (db != nullptr) std::fill(db, db + C, 0.0);
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int64_t start = cu_seqlens[s];
+    for (int64_t t = start; t < cu_seqlens[s + 1]; ++t) {
+      for (int64_t c = 0; c < C; ++c) {
+        const double g = dy[t * C + c];
+        if (db != nullptr) db[c] += g;
+        for (int32_t k = 0; k < K; ++k) {
+          const int64_t src = t - static_cast<int64_t>(dilation) * (K - 1 - k);
+          if (src < start) continue;
+          if (dx != nullptr) dx[src * C + c] += w[c * K + k] * g;
+          if (dw != nullptr) dw[c * K + k] += g * x[src * C + c];
+        }
+      }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

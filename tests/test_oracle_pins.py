@@ -396,3 +396,114 @@ def test_e4m3_spot_values():
     v = synth.bf16_bits_to_f32(oracle.gather_e4m3(np.array([0]), table))[0, :8]
     assert v.tolist() == [1.0, 448.0, 2.0 ** -9, -0.0, -1.0, 2.0 ** -6, 7 * 2.0 ** -9, 0.0]
     assert np.signbit(v[3])
+
+
+# ---------------------------------------------------------------------------
+# segment-aware causal dilated depthwise convolution (PLE layer's short conv):
+# the API page builds it per packed segment as "history zeros ahead of the
+# segment, then its own F.conv1d" (_segmented_conv); torch's conv1d on each
+# zero-padded segment is therefore an independent statement of the same
+# definition
+# ---------------------------------------------------------------------------
+
+def _conv_cases():
+    rng = np.random.default_rng(17)
+    # segments: empty, shorter than the receptive field, one token, long
+    lens = [0, 5, 1, 40, 9, 10, 0, 27]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    for C, K, d in [(3, 4, 3), (5, 1, 1), (2, 4, 1), (4, 3, 5), (1, 8, 2)]:
+        yield rng, cu, C, K, d
+
+
+def _torch_segment_conv(x, cu, w, d, b):
+    import torch
+    out = []
+    K = w.shape[1]
+    for s in range(len(cu) - 1):
+        if cu[s + 1] == cu[s]:
+            continue  # an empty segment has no output rows
+        seg = torch.from_numpy(x[cu[s]:cu[s + 1]]).T[None]  # [1, C, L]
+        seg = torch.nn.functional.pad(seg, ((K - 1) * d, 0))
+        y = torch.nn.functional.conv1d(seg, torch.from_numpy(w)[:, None, :], None if b is None else torch.from_numpy(b),
+                                       dilation=d, groups=w.shape[0])
+        out.append(y[0].T.numpy())
+    return np.concatenate(out) if out else np.zeros((0, x.shape[1]))
+
+
+def test_conv_matches_per_segment_conv1d():
+    for rng, cu, C, K, d in _conv_cases():
+        T = int(cu[-1])
+        x = rng.standard_normal((T, C))
+        w = rng.standard_normal((C, K))
+        b = rng.standard_normal(C)
+        for bias in (None, b):
+            y = oracle.conv_forward(x, cu, w, d, bias)
+            np.testing.assert_allclose(y, _torch_segment_conv(x, cu, w, d, bias), rtol=1e-12, atol=1e-12)
+
+
+def test_conv_closed_forms():
+    rng = np.random.default_rng(3)
+    cu = np.array([0, 7, 7, 20, 21], np.int32)
+    T, C, K, d = 21, 3, 4, 3
+    x = rng.standard_normal((T, C))
+    # only the last tap: the identity
+    w = np.zeros((C, K)); w[:, K - 1] = 1.0
+    np.testing.assert_array_equal(oracle.conv_forward(x, cu, w, d), x)
+    # only tap K-1-m: a shift by m*d inside each segment, zeros at its start
+    for m in range(1, K):
+        w = np.zeros((C, K)); w[:, K - 1 - m] = 1.0
+        want = np.zeros_like(x)
+        for s in range(len(cu) - 1):
+            lo, hi = cu[s], cu[s + 1]
+            if hi - lo > m * d:
+                want[lo + m * d:hi] = x[lo:hi - m * d]
+        np.testing.assert_array_equal(oracle.conv_forward(x, cu, w, d), want)
+    # bias alone
+    b = rng.standard_normal(C)
+    np.testing.assert_array_equal(oracle.conv_forward(x, cu, np.zeros((C, K)), d, b), np.broadcast_to(b, (T, C)))
+
+
+def test_conv_causal_and_segment_local():
+    rng = np.random.default_rng(4)
+    cu = np.array([0, 12, 30], np.int32)
+    x = rng.standard_normal((30, 2))
+    w = rng.standard_normal((2, 4))
+    y = oracle.conv_forward(x, cu, w, 3)
+    x2 = x.copy()
+    x2[20:] += 100.0  # later positions of segment 1
+    y2 = oracle.conv_forward(x2, cu, w, 3)
+    np.testing.assert_array_equal(y2[:20], y[:20])
+    x3 = x.copy()
+    x3[:12] -= 50.0   # all of segment 0
+    y3 = oracle.conv_forward(x3, cu, w, 3)
+    np.testing.assert_array_equal(y3[12:], y[12:])
+
+
+def test_conv_backward_matches_autograd_and_adjoint():
+    import torch
+    for rng, cu, C, K, d in _conv_cases():
+        T = int(cu[-1])
+        x = rng.standard_normal((T, C))
+        w = rng.standard_normal((C, K))
+        dy = rng.standard_normal((T, C))
+        dx, dw, db = oracle.conv_backward(dy, x, cu, w, d)
+        xt = torch.from_numpy(x).requires_grad_(True)
+        wt = torch.from_numpy(w).requires_grad_(True)
+        bt = torch.zeros(C, dtype=torch.float64, requires_grad=True)
+        outs = []
+        for s in range(len(cu) - 1):
+            if cu[s + 1] == cu[s]:
+                continue
+            seg = torch.nn.functional.pad(xt[cu[s]:cu[s + 1]].T[None], ((K - 1) * d, 0))
+            outs.append(torch.nn.functional.conv1d(seg, wt[:, None, :], bt, dilation=d, groups=C)[0].T)
+        (torch.cat(outs) * torch.from_numpy(dy)).sum().backward()
+        np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(dw, wt.grad.numpy(), rtol=1e-12, atol=1e-11)
+        np.testing.assert_allclose(db, bt.grad.numpy(), rtol=1e-12, atol=1e-12)
+        # adjoint identity on integers (exact in fp64): <conv(x), dy> = <x, dx>
+        xi = rng.integers(-8, 9, (T, C)).astype(np.float64)
+        wi = rng.integers(-4, 5, (C, K)).astype(np.float64)
+        gi = rng.integers(-8, 9, (T, C)).astype(np.float64)
+        dxi, dwi, _ = oracle.conv_backward(gi, xi, cu, wi, d)
+        assert float((oracle.conv_forward(xi, cu, wi, d) * gi).sum()) == float((xi * dxi).sum())
+        assert float((oracle.conv_forward(xi, cu, wi, d) * gi).sum()) == float((wi * dwi).sum())
