@@ -236,6 +236,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=8192)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--conv", action="store_true",
+                    help="time the PLE layer's short convolution (forward + backward) instead of the lookup")
+    ap.add_argument("--conv-channels", type=int, default=8192, help="channels of the --conv workload")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -265,6 +268,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
+    if args.conv:
+        return run_conv(args, rank, world, dev, dist)
     w = workload(args.workload, replica_seed(args.seed, rank))
     plan = ple.Plan.from_workload(w)
     T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
@@ -386,7 +391,9 @@ def main():
         if ms_bwd > ms_fwd:
             roofline = bwd_roof
 
-    launches_per_step = 1 + (2 if do_bwd else 0)  # lookup_kernel; sort_kernel (all passes) and the fold kernel
+    # lookup_kernel; the backward: clear, key_hist, one sort_pass per 8-bit digit of the row ids, the fold
+    sort_passes = max(1, (int(w.num_rows).bit_length() + 7) // 8)
+    launches_per_step = 1 + (3 + sort_passes if do_bwd else 0)
     value = world * T_out / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers
@@ -457,6 +464,167 @@ def main():
                 "roofline": roofline, "roofline_fwd": fwd_roof, "roofline_bwd": bwd_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
                 "clocks": clocks, "wall_s_timed_region": wall}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_conv(args, rank, world, dev, dist):
+    """--conv: the PLE layer's short convolution (segment-aware, causal,
+    dilation = ngram_size, K = 4) over the single-layer packing with
+    --conv-channels bf16 channels: one step = ple_conv_forward +
+    ple_conv_backward (dx, dweight, dbias)."""
+    import torch
+
+    import hashed_gram_embedding_ple_b200 as ple
+    import synth
+    from synth import gpu as sgpu
+
+    base = synth.single_layer_bf16(replica_seed(args.seed, rank))
+    cu_np = base.cu_seqlens
+    T, C, K, dil = int(cu_np[-1]), int(args.conv_channels), 4, base.ngram_size
+    seed = 1000 + replica_seed(args.seed, rank)
+    x = torch.empty(T, C, dtype=torch.bfloat16, device=dev)
+    g = torch.empty(T, C, dtype=torch.bfloat16, device=dev)
+    sgpu.fill_(x, seed, 1.0)
+    sgpu.fill_(g, seed + 1, 1.0)
+    gen = torch.Generator().manual_seed(seed)
+    wt = (torch.randn(C, K, generator=gen) * 0.5).to(dev)
+    bt = torch.randn(C, generator=gen).to(dev)
+    cu = torch.from_numpy(cu_np).to(dev)
+    y, dx = torch.empty_like(x), torch.empty_like(x)
+    dw, db = torch.zeros(C, K, device=dev), torch.zeros(C, device=dev)
+    ws = torch.empty(ple.conv_workspace_bytes(T, C, K), dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def flush_l2():
+        flush_w.zero_()
+        flush_r.sum()
+
+    def fwd(xin):
+        ple.conv_forward(xin, cu, wt, dil, bt, out=y)
+
+    def bwd(gin, xin):
+        ple.conv_backward(gin, xin, cu, wt, dil, dx=dx, dweight=dw, dbias=db, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush_l2()
+        fwd(x)
+        bwd(g, x)
+    torch.cuda.synchronize()
+    if ple.ple_status(dev) != ple.PLE_OK:
+        raise SystemExit("libple async status after warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush_l2()
+        ev[k][0].record(stream)
+        fwd(x)
+        ev[k][1].record(stream)
+        bwd(g, x)
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    if ple.ple_status(dev) != ple.PLE_OK:
+        raise SystemExit("libple async status after the timed steps")
+    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
+    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
+    ms_step, ms_fwd, ms_bwd = reduce_max([statistics.mean(a + b for a, b in zip(fwd_ms, bwd_ms)),
+                                          statistics.mean(fwd_ms), statistics.mean(bwd_ms)], dist, dev)
+    peak, peak_kind = measured_peaks()
+    e = 2
+    nchunks = max(1, -(-ws.numel() // (C * (K + 1) * 4)))
+    fwd_bytes = 2 * T * C * e                                     # x read, y written
+    bwd_bytes = 3 * T * C * e + 2 * nchunks * C * (K + 1) * 4    # dy and x read, dx written; partial sums
+    fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
+    bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9
+    src = ["hashed_gram_embedding_ple_b200/csrc/conv.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+    roof_f = {"bound": "hbm", "achieved": fwd_gbs, "peak": peak, "unit": "GB/s", "frac": fwd_gbs / peak,
+              "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": fwd_bytes,
+              "traffic": traffic_from_profiles("conv_forward_conv_single_layer", src), "kernel": "conv_forward_kernel",
+              "peak_source": f"{peak_kind} hbm_gbs"}
+    roof_b = {"bound": "hbm", "achieved": bwd_gbs, "peak": peak, "unit": "GB/s", "frac": bwd_gbs / peak,
+              "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": bwd_bytes,
+              "traffic": traffic_from_profiles("conv_backward_conv_single_layer", src),
+              "kernel": "conv_backward_kernel + conv_reduce_kernel", "peak_source": f"{peak_kind} hbm_gbs"}
+    roofline = roof_b if ms_bwd > ms_fwd else roof_f
+
+    e2e = None
+    if args.e2e_steps > 0:
+        hx, hg = x.cpu().pin_memory(), g.cpu().pin_memory()
+        hy, hdx = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
+        dxin, dgin = torch.empty_like(x), torch.empty_like(g)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for k in range(args.e2e_steps + 1):
+            flush_l2()
+            e0.record(stream)
+            dxin.copy_(hx, non_blocking=True)
+            dgin.copy_(hg, non_blocking=True)
+            fwd(dxin)
+            bwd(dgin, dxin)
+            hy.copy_(y, non_blocking=True)
+            hdx.copy_(dx, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if k >= 1:
+                times.append(e0.elapsed_time(e1))
+        (t_e2e,) = reduce_max([statistics.mean(times)], dist, dev)
+        e2e = {"value": world * T / (t_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 2 * T * C * e,
+               "d2h_bytes_per_step": 2 * T * C * e, "ms_per_step": t_e2e,
+               "what": "pinned H2D of x and dy, ple_conv_forward, ple_conv_backward, D2H of y and dx"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        sample = min(T, 1024)
+        cu_s = np.asarray([c for c in cu_np if c < sample] + [sample], np.int32)
+        xs = torch_to_np(x[:sample]).view(np.uint16)
+        gs = torch_to_np(g[:sample]).view(np.uint16)
+        xf = synth.bf16_bits_to_f32(xs).astype(np.float64)
+        gf = synth.bf16_bits_to_f32(gs).astype(np.float64)
+        wn, bn = wt.cpu().numpy().astype(np.float64), bt.cpu().numpy().astype(np.float64)
+        tot_t, tot_s, reps = 0, 0.0, 0
+        while tot_s < args.cpu_seconds and reps < 500:
+            t0 = time.perf_counter()
+            oracle.conv_forward(xf, cu_s, wn, dil, bn)
+            oracle.conv_backward(gf, xf, cu_s, wn, dil)
+            tot_s += time.perf_counter() - t0
+            tot_t += sample
+            reps += 1
+        cpu = {"value": tot_t / tot_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{reps} passes over the first {sample} tokens x {C} channels (forward + backward, fp64 "
+                         f"scalar loops, one thread), {tot_s:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": "PLE short conv tokens/s and achieved HBM GB/s (fwd, bwd) vs 8 TB/s", "value":
+                world * T / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 activations, f32 weights and accumulation", "data": "synthetic",
+                "config": {"workload": "conv_single_layer", "tokens": T, "sequences": int(len(cu_np) - 1),
+                           "channels": C, "kernel_size": K, "dilation": dil, "parallelism": f"replicas{world}",
+                           "l2": "flushed between steps (512 MB written, then another 512 MB read); outside the events",
+                           "step": "ple_conv_forward + ple_conv_backward (dx, dweight, dbias)"},
+                "fwd": {"ms": ms_fwd, "gb_per_s": fwd_gbs, "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS,
+                        "frac_of_measured": fwd_gbs / peak},
+                "bwd": {"ms": ms_bwd, "gb_per_s": bwd_gbs, "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS,
+                        "frac_of_measured": bwd_gbs / peak},
+                "roofline": roofline, "roofline_fwd": roof_f, "roofline_bwd": roof_b, "cpu_baseline": cpu,
+                "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks, "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

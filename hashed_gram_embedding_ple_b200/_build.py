@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libple.so")
-SOURCES = ["plan.cu", "lookup.cu", "grad.cu"]
+SOURCES = ["plan.cu", "lookup.cu", "grad.cu", "conv.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -37,8 +37,9 @@ _DTYPE_OF_CODE = {PLE_F32: torch.float32, PLE_BF16: torch.bfloat16, PLE_F8E4M3: 
 EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_lookup_slice",
            "ple_gather",
            "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic",
-           "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_status",
-           "ple_strerror", "ple_last_cuda_error")
+           "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_conv_forward",
+           "ple_conv_backward_workspace_bytes", "ple_conv_backward", "ple_status", "ple_strerror",
+           "ple_last_cuda_error")
 
 
 class PleError(RuntimeError):
@@ -84,13 +85,18 @@ def _lib():
         lib.ple_grad_scatter_noalloc.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
         lib.ple_grad_scatter_noalloc_scratch_bytes.argtypes = []
         lib.ple_grad_scatter_noalloc_scratch_bytes.restype = sz
+        lib.ple_conv_forward.argtypes = [vp, ctypes.c_int, i64, i64, vp, i32, vp, i32, i32, vp, vp, vp]
+        lib.ple_conv_backward_workspace_bytes.argtypes = [i64, i64, i32]
+        lib.ple_conv_backward_workspace_bytes.restype = sz
+        lib.ple_conv_backward.argtypes = [vp, vp, ctypes.c_int, i64, i64, vp, i32, vp, i32, i32, vp, vp, vp, vp, sz,
+                                          vp]
         lib.ple_status.argtypes = [vp]
         lib.ple_strerror.argtypes = [ctypes.c_int]
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
         for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_lookup_slice", "ple_gather", "ple_grad_scatter",
-                     "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_status",
-                     "ple_last_cuda_error"):
+                     "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_conv_forward",
+                     "ple_conv_backward", "ple_status", "ple_last_cuda_error"):
             getattr(lib, name).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -317,6 +323,66 @@ def ple_grad_scatter_noalloc(plan: Plan, rows, grad_out, table_grad):
     _check(_lib().ple_grad_scatter_noalloc(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
                                            _stream(rows.device)), "ple_grad_scatter_noalloc")
     return table_grad
+
+
+# ---------------------------------------------------------------------------
+# the PLE layer's short convolution (segment-aware, causal, dilated, depthwise)
+# ---------------------------------------------------------------------------
+
+def _conv_check(x, cu_seqlens, weight):
+    if x.dim() != 2 or x.dtype not in _DTYPES or not x.is_contiguous() or not x.is_cuda:
+        raise ValueError("x must be a contiguous [tokens, channels] float32 or bfloat16 CUDA tensor")
+    _as_i32(cu_seqlens, "cu_seqlens")
+    if weight.dtype != torch.float32 or not weight.is_contiguous() or weight.dim() != 2 \
+            or weight.shape[0] != x.shape[1] or not weight.is_cuda:
+        raise ValueError("weight must be a contiguous float32 CUDA tensor [channels, kernel_size]")
+
+
+def conv_forward(x, cu_seqlens, weight, dilation: int, bias=None, out=None):
+    """y = segment-aware causal dilated depthwise convolution of x [T, C] with
+    weight [C, K] (+ bias [C]); y has x's shape and dtype."""
+    _conv_check(x, cu_seqlens, weight)
+    T, C = x.shape
+    if bias is not None and (bias.dtype != torch.float32 or bias.numel() != C or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous float32 tensor [channels]")
+    if out is None:
+        out = torch.empty_like(x)
+    elif out.shape != x.shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError("out must match x")
+    _check(_lib().ple_conv_forward(_ptr(x), _DTYPES[x.dtype], T, C, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                   _ptr(weight), weight.shape[1], int(dilation), _ptr(bias), _ptr(out),
+                                   _stream(x.device)), "ple_conv_forward")
+    return out
+
+
+def conv_workspace_bytes(num_tokens: int, channels: int, kernel_size: int) -> int:
+    return int(_lib().ple_conv_backward_workspace_bytes(int(num_tokens), int(channels), int(kernel_size)))
+
+
+def conv_backward(dy, x, cu_seqlens, weight, dilation: int, dx=None, want_dx: bool = True, dweight=None,
+                  dbias=None, workspace=None):
+    """Gradients of conv_forward: returns (dx, dweight, dbias).  dx is
+    written (allocated unless given; skipped with want_dx=False); dweight
+    [C, K] and dbias [C] are fp32 tensors accumulated into when given."""
+    _conv_check(x, cu_seqlens, weight)
+    if dy.shape != x.shape or dy.dtype != x.dtype or not dy.is_contiguous():
+        raise ValueError("dy must match x")
+    T, C = x.shape
+    K = weight.shape[1]
+    if dx is None and want_dx:
+        dx = torch.empty_like(x)
+    elif dx is not None and (dx.shape != x.shape or dx.dtype != x.dtype or not dx.is_contiguous()):
+        raise ValueError("dx must match x")
+    for name, t, n in (("dweight", dweight, C * K), ("dbias", dbias, C)):
+        if t is not None and (t.dtype != torch.float32 or t.numel() != n or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of {n} elements")
+    if (dweight is not None or dbias is not None) and workspace is None:
+        workspace = torch.empty(max(conv_workspace_bytes(T, C, K), 1), dtype=torch.uint8, device=x.device)
+    _check(_lib().ple_conv_backward(_ptr(dy), _ptr(x), _DTYPES[x.dtype], T, C, _ptr(cu_seqlens),
+                                    cu_seqlens.numel() - 1, _ptr(weight), K, int(dilation), _ptr(dx), _ptr(dweight),
+                                    _ptr(dbias), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                    _stream(x.device)), "ple_conv_backward")
+    return dx, dweight, dbias
 
 
 def noalloc_scratch_bytes() -> int:

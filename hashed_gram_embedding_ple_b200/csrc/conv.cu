@@ -1,0 +1,431 @@
+// The PLE layer's short convolution: a causal, dilated, depthwise 1-D
+// convolution over packed tokens in which every packed segment starts with
+// zero history (Qwen3_8_FlashNextPLELayer._causal_short_conv and
+// _segmented_conv, NeMo AutoModel engram API page):
+//   y[t, c] = bias[c] + sum_k w[c, k] * x[t - dilation*(K-1-k), c],
+// a tap before the first position of t's segment reading zero.
+//
+// HBM-bound: x is read once from DRAM and y written once.  A thread owns one
+// 16-byte vector of channels (8 bf16 or 4 fp32) and walks a chunk of tokens
+// one residue class modulo the dilation at a time (the taps of a token lie
+// in its class), keeping the class's previous rows in registers, so every
+// load and store of a warp covers 512 consecutive bytes of a token row and
+// each row is loaded once (plus K-1 rows of history per class and chunk).
+// The backward pass computes dx (the same taps looking ahead, inside the
+// segment) and, in the same sweep, per-chunk partial sums of dw and db; a
+// second kernel adds the chunk partials in chunk order (deterministic) and
+// adds the result once into the caller's dw and db.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace ple {
+namespace {
+
+constexpr int kConvThreads = 128;     // channel vectors per block
+constexpr int kConvChunk = 128;       // tokens per block, forward
+constexpr int kConvBwdChunk = 256;    // least tokens per block, backward
+constexpr int64_t kMaxPartials = 1024;  // at most this many backward chunks (their partial sums)
+constexpr int kMaxTaps = 8;
+
+template <bool BF16>
+struct Vec {
+  static constexpr int n = BF16 ? 8 : 4;  // channels per 16-byte vector
+};
+
+template <bool BF16>
+__device__ __forceinline__ void unpack(const uint4& u, float* v) {
+  if constexpr (BF16) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint4 pack(const float* v) {
+  if constexpr (BF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);  // .x = low half
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+  }
+}
+
+__device__ __forceinline__ uint4 ld_vec(const unsigned char* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+// The packed segment of the positions a thread walks (in increasing order).
+// Bounds are clamped to [0, T]; with a malformed cu_seqlens (flagged by
+// check_cu) a position the array does not cover is treated as a segment of
+// its own, so every access stays inside the tensors.
+struct Segment {
+  const int32_t* cu;
+  int32_t num_seqs, s;
+  int64_t T, lo, hi;
+  __device__ void load() {
+    lo = min(max(static_cast<int64_t>(__ldg(cu + s)), int64_t{0}), T);
+    hi = min(max(static_cast<int64_t>(__ldg(cu + s + 1)), int64_t{0}), T);
+  }
+  __device__ void start(int64_t t) {  // the last s with cu[s] <= t (binary search)
+    int32_t a = 0, b = num_seqs - 1;
+    while (a < b) {
+      const int32_t mid = (a + b + 1) >> 1;
+      if (static_cast<int64_t>(__ldg(cu + mid)) <= t) a = mid; else b = mid - 1;
+    }
+    s = a;
+    load();
+  }
+  __device__ void advance(int64_t t) {  // to the segment holding t (empty segments skipped)
+    while (t >= hi && s + 1 < num_seqs) {
+      ++s;
+      load();
+    }
+  }
+  __device__ int64_t first(int64_t t) const { return t >= lo && t < hi ? lo : t; }    // history starts here
+  __device__ int64_t end(int64_t t) const { return t >= lo && t < hi ? hi : t + 1; }  // lookahead ends here
+};
+
+// Block (0, 0) checks cu_seqlens once per launch: cu[0] == 0, cu[S] == T,
+// non-decreasing.  Bad input only raises a flag.
+__device__ void check_cu(const int32_t* __restrict__ cu, int32_t num_seqs, int64_t T, unsigned int* status) {
+  if (blockIdx.x != 0 || blockIdx.y != 0) return;
+  bool bad = false;
+  if (threadIdx.x == 0) bad = (cu[0] != 0) || (static_cast<int64_t>(cu[num_seqs]) != T);
+  for (int32_t i = threadIdx.x; i < num_seqs; i += blockDim.x) bad |= cu[i + 1] < cu[i];
+  if (bad) raise_flag(status, PLE_ERR_BAD_SEQLENS);
+}
+
+// Forward.  Block (token chunk bx, vector block by); thread = one channel
+// vector.  The taps of token t lie at t, t - d, ..., t - (K-1) d: all in
+// t's residue class modulo the dilation d.  So a thread walks the chunk one
+// residue class (chain) at a time, K chain steps per iteration, holding the
+// chain's previous K rows in registers (static indices): one new row load
+// per output, K of them in flight; the K-1 rows before the chunk come from
+// one load each at the start of every chain.
+template <bool BF16, int K>
+__global__ void __launch_bounds__(kConvThreads)
+conv_forward_kernel(const unsigned char* __restrict__ x, int64_t T, int64_t nvec, const int32_t* __restrict__ cu,
+                    int32_t num_seqs, const float* __restrict__ w, int dilation,
+                    const float* __restrict__ bias, unsigned char* __restrict__ y, unsigned int* status) {
+  constexpr int V = Vec<BF16>::n;
+  check_cu(cu, num_seqs, T, status);
+  const int64_t cv = static_cast<int64_t>(blockIdx.y) * kConvThreads + threadIdx.x;  // channel vector
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kConvChunk;
+  if (cv >= nvec || t0 >= T) return;
+  const int64_t C = nvec * V, row = C * (BF16 ? 2 : 4);
+  float wr[V][K], b[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    b[v] = bias != nullptr ? __ldg(bias + cv * V + v) : 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) wr[v][k] = __ldg(w + (cv * V + v) * K + k);
+  }
+  const int64_t t1 = min(T, t0 + kConvChunk), d = dilation;
+  const unsigned char* xc = x + cv * 16;
+  unsigned char* yc = y + cv * 16;
+  Segment sg{cu, num_seqs, 0, T, 0, 0};
+  for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
+    sg.start(t0 + r);
+    uint4 prev[K], cur[K];  // chain rows: prev = the K steps before cur
+#pragma unroll
+    for (int j = 1; j < K; ++j) {  // steps -1 .. -(K-1) before the chain's first token
+      const int64_t t = t0 + r - static_cast<int64_t>(K - j) * d;
+      prev[j] = t >= 0 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+    }
+    for (int64_t tb = t0 + r; tb < t1; tb += K * d) {
+#pragma unroll
+      for (int m = 0; m < K; ++m) {
+        const int64_t t = tb + m * d;
+        cur[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int m = 0; m < K; ++m) {
+        const int64_t t = tb + m * d;
+        if (t < t1) {
+          sg.advance(t);
+          const int64_t seg_lo = sg.first(t);
+          float acc[V];
+#pragma unroll
+          for (int v = 0; v < V; ++v) acc[v] = b[v];
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const int j = K - 1 - k;  // chain steps back
+            if (t - j * d >= seg_lo) {  // before the segment: zero history
+              float xv[V];
+              unpack<BF16>(m - j >= 0 ? cur[m - j] : prev[K + m - j], xv);
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], xv[v], acc[v]);
+            }
+          }
+          st_cs(yc + t * row, pack<BF16>(acc));
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < K; ++m) prev[m] = cur[m];
+    }
+  }
+}
+
+// Backward sweep: dx (nullable) and this chunk's partial sums of dw and db,
+// written to part[chunk][c][K + 1] (tap k at k, the bias at K).  The same
+// residue chains as the forward: output t took x at chain steps 0..K-1 back
+// (dw), and x[t] fed the outputs at chain steps 0..K-1 ahead (dx).  Per K
+// chain steps a thread loads K rows of x (the current steps) and K rows of
+// dy (K steps ahead); the rest comes from the previous iteration's registers.
+template <bool BF16, int K>
+__global__ void __launch_bounds__(kConvThreads)
+conv_backward_kernel(const unsigned char* __restrict__ dy, const unsigned char* __restrict__ x, int64_t T,
+                     int64_t nvec, const int32_t* __restrict__ cu, int32_t num_seqs, const float* __restrict__ w,
+                     int dilation, int64_t chunk, unsigned char* __restrict__ dx, float* __restrict__ part,
+                     unsigned int* status) {
+  constexpr int V = Vec<BF16>::n;
+  check_cu(cu, num_seqs, T, status);
+  const int64_t cv = static_cast<int64_t>(blockIdx.y) * kConvThreads + threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  if (cv >= nvec) return;
+  const int64_t C = nvec * V, row = C * (BF16 ? 2 : 4);
+  float wr[V][K], gw[V][K], gb[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    gb[v] = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      wr[v][k] = __ldg(w + (cv * V + v) * K + k);
+      gw[v][k] = 0.f;
+    }
+  }
+  const int64_t t1 = min(T, t0 + chunk), d = dilation;
+  const unsigned char* xc = x + cv * 16;
+  const unsigned char* gc = dy + cv * 16;
+  Segment sg{cu, num_seqs, 0, T, 0, 0};
+  // each chain's tokens in ascending order, chains in ascending residue: the
+  // order of the partial sums (a fixed function of the sizes)
+  for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
+    sg.start(t0 + r);
+    uint4 xp[K], xn[K], gn[K], ga[K];  // x: previous / current steps; dy: current / K steps ahead
+#pragma unroll
+    for (int j = 1; j < K; ++j) {
+      const int64_t t = t0 + r - static_cast<int64_t>(K - j) * d;
+      xp[j] = t >= 0 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int m = 0; m < K; ++m) {
+      const int64_t t = t0 + r + m * d;
+      gn[m] = t < T ? ld_vec(gc + t * row) : make_uint4(0, 0, 0, 0);
+    }
+    for (int64_t tb = t0 + r; tb < t1; tb += K * d) {
+#pragma unroll
+      for (int m = 0; m < K; ++m) {
+        const int64_t t = tb + m * d, ta = t + K * d;
+        xn[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+        ga[m] = ta < T && t < t1 ? ld_vec(gc + ta * row) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int m = 0; m < K; ++m) {
+        const int64_t t = tb + m * d;
+        if (t < t1) {
+          sg.advance(t);
+          const int64_t seg_lo = sg.first(t), seg_hi = sg.end(t);
+          float g[V];
+          unpack<BF16>(gn[m], g);
+#pragma unroll
+          for (int v = 0; v < V; ++v) gb[v] += g[v];
+          float acc[V];
+#pragma unroll
+          for (int v = 0; v < V; ++v) acc[v] = 0.f;
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const int j = K - 1 - k;  // chain steps
+            if (t - j * d >= seg_lo) {  // output t read x[t - j d] through tap k
+              float xv[V];
+              unpack<BF16>(m - j >= 0 ? xn[m - j] : xp[K + m - j], xv);
+#pragma unroll
+              for (int v = 0; v < V; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
+            }
+            if (dx != nullptr && t + j * d < seg_hi) {  // x[t] fed output t + j d through tap k
+              float gv[V];
+              unpack<BF16>(m + j < K ? gn[m + j] : ga[m + j - K], gv);
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+            }
+          }
+          if (dx != nullptr) st_cs(dx + t * row + cv * 16, pack<BF16>(acc));
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < K; ++m) {
+        xp[m] = xn[m];
+        gn[m] = ga[m];
+      }
+    }
+  }
+  if (part == nullptr) return;  // dx only
+  float* pc = part + static_cast<int64_t>(blockIdx.x) * C * (K + 1);
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const int64_t c = cv * V + v;
+#pragma unroll
+    for (int k = 0; k < K; ++k) pc[c * (K + 1) + k] = gw[v][k];
+    pc[c * (K + 1) + K] = gb[v];
+  }
+}
+
+// dw[c, k] += sum over chunks (in chunk order) of the partials; db likewise.
+__global__ void conv_reduce_kernel(const float* __restrict__ part, int64_t nchunks, int64_t C, int K,
+                                   float* __restrict__ dw, float* __restrict__ db) {
+  const int64_t n = C * (K + 1);
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  wait_for_prior_grid();
+  float sum = part[e];
+  for (int64_t q = 1; q < nchunks; ++q) sum += part[q * n + e];
+  const int64_t c = e / (K + 1);
+  const int k = static_cast<int>(e - c * (K + 1));
+  if (k < K) {
+    if (dw != nullptr) dw[c * K + k] += sum;
+  } else if (db != nullptr) {
+    db[c] += sum;
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ple_status_t check_conv_args(const void* x, ple_dtype_t dtype, int64_t T, int64_t C, const int32_t* cu,
+                             int32_t S, const float* w, int32_t K, int32_t dilation) {
+  if (T < 0 || C < 1 || K < 1 || dilation < 1) return PLE_ERR_INVALID_ARG;
+  if (dtype != PLE_F32 && dtype != PLE_BF16) return PLE_ERR_INVALID_ARG;
+  if (K > kMaxTaps) return PLE_ERR_UNSUPPORTED;
+  if (T == 0) return PLE_OK;
+  if (x == nullptr || cu == nullptr || w == nullptr || S < 1) return PLE_ERR_INVALID_ARG;
+  if (T > (int64_t{1} << 40) || C > (int64_t{1} << 24)) return PLE_ERR_UNSUPPORTED;
+  if ((C * (dtype == PLE_F32 ? 4 : 2)) % 16 != 0 || !aligned16(x)) return PLE_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(cu) & 3u) != 0 || (reinterpret_cast<uintptr_t>(w) & 3u) != 0)
+    return PLE_ERR_ALIGNMENT;
+  return PLE_OK;
+}
+
+// tokens per backward block: at least kConvBwdChunk, and few enough blocks
+// along the tokens that at most kMaxPartials partial sums are kept
+int64_t conv_chunk_bwd(int64_t T) {
+  const int64_t need = (T + kMaxPartials - 1) / kMaxPartials;
+  return need > kConvBwdChunk ? need : kConvBwdChunk;
+}
+int64_t conv_chunks_bwd(int64_t T) {
+  const int64_t c = conv_chunk_bwd(T);
+  return (T + c - 1) / c;
+}
+
+}  // namespace
+}  // namespace ple
+
+using namespace ple;
+
+extern "C" {
+
+ple_status_t ple_conv_forward(const void* x, ple_dtype_t dtype, int64_t T, int64_t C, const int32_t* cu_seqlens,
+                              int32_t num_seqs, const float* weight, int32_t K, int32_t dilation, const float* bias,
+                              void* y, void* stream) {
+  ple_status_t st = check_conv_args(x, dtype, T, C, cu_seqlens, num_seqs, weight, K, dilation);
+  if (st != PLE_OK || T == 0) return st;
+  if (y == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned16(y) || (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u) != 0)) return PLE_ERR_ALIGNMENT;
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const bool bf = dtype == PLE_BF16;
+  const int64_t nvec = C / (bf ? 8 : 4);
+  // grid.x: token chunks (T <= 2^40 keeps them < 2^31); grid.y: channel blocks (C <= 2^24 keeps them <= 32768)
+  const dim3 grid(static_cast<unsigned>((T + kConvChunk - 1) / kConvChunk),
+                  static_cast<unsigned>((nvec + kConvThreads - 1) / kConvThreads));
+  const auto s = static_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const unsigned char*>(x);
+  auto* yb = static_cast<unsigned char*>(y);
+#define PLE_CONV_FWD(KK)                                                                                    \
+  case KK:                                                                                                  \
+    if (bf)                                                                                                 \
+      conv_forward_kernel<true, KK><<<grid, kConvThreads, 0, s>>>(xb, T, nvec, cu_seqlens, num_seqs, weight, \
+                                                                   dilation, bias, yb, status);             \
+    else                                                                                                    \
+      conv_forward_kernel<false, KK><<<grid, kConvThreads, 0, s>>>(xb, T, nvec, cu_seqlens, num_seqs, weight, \
+                                                                    dilation, bias, yb, status);            \
+    break;
+  switch (K) {
+    PLE_CONV_FWD(1) PLE_CONV_FWD(2) PLE_CONV_FWD(3) PLE_CONV_FWD(4)
+    PLE_CONV_FWD(5) PLE_CONV_FWD(6) PLE_CONV_FWD(7) PLE_CONV_FWD(8)
+    default: return PLE_ERR_UNSUPPORTED;
+  }
+#undef PLE_CONV_FWD
+  return check_launch();
+}
+
+size_t ple_conv_backward_workspace_bytes(int64_t T, int64_t C, int32_t K) {
+  if (T <= 0 || C < 1 || K < 1 || K > kMaxTaps) return 0;
+  return static_cast<size_t>(conv_chunks_bwd(T)) * static_cast<size_t>(C) * static_cast<size_t>(K + 1) *
+         sizeof(float);
+}
+
+ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype, int64_t T, int64_t C,
+                               const int32_t* cu_seqlens, int32_t num_seqs, const float* weight, int32_t K,
+                               int32_t dilation, void* dx, float* dweight, float* dbias, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  ple_status_t st = check_conv_args(x, dtype, T, C, cu_seqlens, num_seqs, weight, K, dilation);
+  if (st != PLE_OK || T == 0) return st;
+  if (dy == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned16(dy) || (dx != nullptr && !aligned16(dx))) return PLE_ERR_ALIGNMENT;
+  const bool want_params = dweight != nullptr || dbias != nullptr;
+  if (want_params) {
+    if (workspace == nullptr || workspace_bytes < ple_conv_backward_workspace_bytes(T, C, K))
+      return PLE_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return PLE_ERR_ALIGNMENT;
+  } else if (dx == nullptr) {
+    return PLE_OK;  // nothing asked for
+  }
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const bool bf = dtype == PLE_BF16;
+  const int64_t nvec = C / (bf ? 8 : 4);
+  const int64_t chunk = conv_chunk_bwd(T), nchunks = conv_chunks_bwd(T);
+  const dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>((nvec + kConvThreads - 1) / kConvThreads));
+  const auto s = static_cast<cudaStream_t>(stream);
+  float* part = want_params ? static_cast<float*>(workspace) : nullptr;  // partial sums only when asked for
+  const auto* g = static_cast<const unsigned char*>(dy);
+  const auto* xb = static_cast<const unsigned char*>(x);
+  auto* dxb = static_cast<unsigned char*>(dx);
+#define PLE_CONV_BWD(KK)                                                                                     \
+  case KK:                                                                                                   \
+    if (bf)                                                                                                  \
+      conv_backward_kernel<true, KK><<<grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs, weight, \
+                                                                    dilation, chunk, dxb, part, status);      \
+    else                                                                                                     \
+      conv_backward_kernel<false, KK><<<grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs,      \
+                                                                     weight, dilation, chunk, dxb, part, status); \
+    break;
+  switch (K) {
+    PLE_CONV_BWD(1) PLE_CONV_BWD(2) PLE_CONV_BWD(3) PLE_CONV_BWD(4)
+    PLE_CONV_BWD(5) PLE_CONV_BWD(6) PLE_CONV_BWD(7) PLE_CONV_BWD(8)
+    default: return PLE_ERR_UNSUPPORTED;
+  }
+#undef PLE_CONV_BWD
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (want_params) {
+    const int64_t n = C * (K + 1);
+    e = launch_after(conv_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s,
+                     static_cast<const float*>(part), nchunks, C, static_cast<int>(K), dweight, dbias);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return check_launch();
+}
+
+}  // extern "C"

@@ -191,6 +191,51 @@ ple_status_t ple_grad_scatter_noalloc(const ple_plan_t* plan, const int64_t* row
 /* Bytes of the fixed scratch area ple_grad_scatter_noalloc works in. */
 size_t ple_grad_scatter_noalloc_scratch_bytes(void);
 
+/* ---- The PLE layer's short convolution --------------------------------------
+ * Segment-aware causal dilated depthwise convolution over packed tokens
+ * (Qwen3_8_FlashNextPLELayer._causal_short_conv and _segmented_conv, NeMo
+ * AutoModel engram API page; conv_kernel_size K, default 4, and
+ * short_conv_dilation = ngram_size): every packed segment is convolved as if
+ * it started a fresh row, with (K-1)*dilation zeros of history ahead of it:
+ *   y[t, c] = bias[c] + sum_{k=0}^{K-1} w[c, k] * x[t - dilation*(K-1-k), c],
+ * a tap before the first position of t's segment reading zero.
+ * x, y: [num_tokens, channels] row-major, dtype PLE_BF16 or PLE_F32 (both the
+ * same), 16-byte aligned, channels * element size a multiple of 16 bytes;
+ * weight fp32 [channels, K] (the depthwise Conv1d weight [C, 1, K]);
+ * bias fp32 [channels] or NULL.  Arithmetic in fp32 (one fused multiply-add
+ * per tap, taps in ascending k after the bias), rounded to the output type.
+ * cu_seqlens int32 [num_seqs + 1] as for ple_lookup.  num_tokens == 0 is a
+ * no-op.  Errors: PLE_ERR_INVALID_ARG (null pointer, K < 1, dilation < 1,
+ * other dtype), PLE_ERR_UNSUPPORTED (K > 8, channels > 2^24), PLE_ERR_ALIGNMENT,
+ * PLE_ERR_CUDA; async PLE_ERR_BAD_SEQLENS (outputs still written, every
+ * access inside the tensors). */
+ple_status_t ple_conv_forward(const void* x, ple_dtype_t dtype, int64_t num_tokens, int64_t channels,
+                              const int32_t* cu_seqlens, int32_t num_seqs, const float* weight, int32_t kernel_size,
+                              int32_t dilation, const float* bias, void* y, void* stream);
+
+/* Workspace bytes ple_conv_backward needs for dweight / dbias (0 for 0 tokens). */
+size_t ple_conv_backward_workspace_bytes(int64_t num_tokens, int64_t channels, int32_t kernel_size);
+
+/* Gradients of ple_conv_forward for the output gradient dy (same layout and
+ * dtype as x):
+ *   dx[t, c] = sum_k w[c, k] * dy[t + dilation*(K-1-k), c] over taps that stay
+ *              inside t's segment (overwritten; NULL to skip);
+ *   dweight[c, k] += sum_t dy[t, c] * x[t - dilation*(K-1-k), c] (taps inside
+ *              the segment), dbias[c] += sum_t dy[t, c] (fp32, accumulated
+ *              into; NULL to skip).
+ * The sums over tokens have a fixed order, so results are bit-identical run
+ * to run: the tokens are cut into consecutive chunks (at least 256 tokens,
+ * at most 1024 chunks); each chunk's sum starts from +0 and adds its tokens
+ * in order (fused multiply-add for dweight); the chunk sums are added in
+ * chunk order starting from the first; one final add into dweight / dbias.
+ * workspace (16-byte aligned, ple_conv_backward_workspace_bytes) is needed
+ * only for dweight or dbias.  Errors as ple_conv_forward, plus
+ * PLE_ERR_WORKSPACE. */
+ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype, int64_t num_tokens, int64_t channels,
+                               const int32_t* cu_seqlens, int32_t num_seqs, const float* weight, int32_t kernel_size,
+                               int32_t dilation, void* dx, float* dweight, float* dbias, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, then return and clear the async status word of the
  * current device (PLE_OK if no kernel flagged anything; otherwise the
  * lowest-numbered flagged error).  The word is shared by all plans and

@@ -131,3 +131,34 @@ def test_strerror_covers_codes():
     for c in range(9):
         assert lib.ple_strerror(c)
     assert b"unknown" in lib.ple_strerror(99)
+
+
+def test_conv_rejects_bad_arguments_on_host():
+    lib = ple.lib()
+    f, b = lib.ple_conv_forward, lib.ple_conv_backward
+    BF = binding.PLE_BF16
+    # empty input is a no-op
+    assert f(None, BF, 0, 8, None, 0, None, 4, 3, None, None, None) == 0
+    # bad sizes / kinds
+    assert f(0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 0, 3, None, 0x4000, None) == binding.PLE_ERR_INVALID_ARG
+    assert f(0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 0, None, 0x4000, None) == binding.PLE_ERR_INVALID_ARG
+    assert f(0x1000, 7, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, 0x4000, None) == binding.PLE_ERR_INVALID_ARG
+    assert f(0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 9, 3, None, 0x4000, None) == binding.PLE_ERR_UNSUPPORTED
+    assert f(0x1000, BF, 5, 8, None, 1, 0x3000, 4, 3, None, 0x4000, None) == binding.PLE_ERR_INVALID_ARG
+    assert f(0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, None, None) == binding.PLE_ERR_INVALID_ARG
+    # alignment: 8-byte rows, misaligned x / y
+    assert f(0x1000, BF, 5, 4, 0x2000, 1, 0x3000, 4, 3, None, 0x4000, None) == binding.PLE_ERR_ALIGNMENT
+    assert f(0x1008, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, 0x4000, None) == binding.PLE_ERR_ALIGNMENT
+    assert f(0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, 0x4008, None) == binding.PLE_ERR_ALIGNMENT
+    # backward: parameter gradients need the workspace
+    need = lib.ple_conv_backward_workspace_bytes(5, 8, 4)
+    assert need >= 5 * 8 * 4 * 0 + 8 * 5 * 4
+    assert b(0x5000, 0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, 0x6000, None, None, 0, None) == \
+        binding.PLE_ERR_WORKSPACE
+    assert b(0x5000, 0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, 0x6000, None, 0x7000, need - 1, None) == \
+        binding.PLE_ERR_WORKSPACE
+    assert b(0x5000, 0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, None, None, None, None, 0, None) == 0  # nothing asked
+    assert b(0x5008, 0x1000, BF, 5, 8, 0x2000, 1, 0x3000, 4, 3, 0x8000, None, None, None, 0, None) == \
+        binding.PLE_ERR_ALIGNMENT
+    # 1024 chunks at most: the workspace stops growing with the token count past 256 K tokens
+    assert lib.ple_conv_backward_workspace_bytes(1 << 24, 8, 4) == 1024 * 8 * 5 * 4
