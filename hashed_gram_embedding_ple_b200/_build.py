@@ -11,13 +11,13 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libple.so")
-SOURCES = ["plan.cu", "lookup.cu", "grad.cu", "conv.cu"]
+SOURCES = ["plan.cu", "lookup.cu", "grad.cu", "conv.cu", "host_tier.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES]
-    files += [os.path.join(CSRC, "common.cuh"), os.path.join(INCLUDE, "ple.h")]
+    files += [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "sort.cuh"), os.path.join(INCLUDE, "ple.h")]
     return files
 
 

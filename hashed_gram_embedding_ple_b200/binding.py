@@ -37,7 +37,8 @@ _DTYPE_OF_CODE = {PLE_F32: torch.float32, PLE_BF16: torch.bfloat16, PLE_F8E4M3: 
 EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_lookup_slice",
            "ple_gather",
            "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic",
-           "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_conv_forward",
+           "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_prefetch_workspace_bytes",
+           "ple_prefetch", "ple_gather_cache", "ple_grad_scatter_cache", "ple_conv_forward",
            "ple_conv_backward_workspace_bytes", "ple_conv_backward", "ple_status", "ple_strerror",
            "ple_last_cuda_error")
 
@@ -85,6 +86,11 @@ def _lib():
         lib.ple_grad_scatter_noalloc.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
         lib.ple_grad_scatter_noalloc_scratch_bytes.argtypes = []
         lib.ple_grad_scatter_noalloc_scratch_bytes.restype = sz
+        lib.ple_prefetch_workspace_bytes.argtypes = [vp, i64]
+        lib.ple_prefetch_workspace_bytes.restype = sz
+        lib.ple_prefetch.argtypes = [vp, vp, i64, vp, i32, vp, vp, i64, vp, vp, vp, vp, sz, vp]
+        lib.ple_gather_cache.argtypes = [vp, vp, i64, vp, i64, vp, vp]
+        lib.ple_grad_scatter_cache.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, i64, vp, sz, vp]
         lib.ple_conv_forward.argtypes = [vp, ctypes.c_int, i64, i64, vp, i32, vp, i32, i32, vp, vp, vp]
         lib.ple_conv_backward_workspace_bytes.argtypes = [i64, i64, i32]
         lib.ple_conv_backward_workspace_bytes.restype = sz
@@ -95,7 +101,8 @@ def _lib():
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
         for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_lookup_slice", "ple_gather", "ple_grad_scatter",
-                     "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_conv_forward",
+                     "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_prefetch", "ple_gather_cache",
+                     "ple_grad_scatter_cache", "ple_conv_forward",
                      "ple_conv_backward", "ple_status", "ple_last_cuda_error"):
             getattr(lib, name).restype = ctypes.c_int
         _LIB = lib
@@ -323,6 +330,76 @@ def ple_grad_scatter_noalloc(plan: Plan, rows, grad_out, table_grad):
     _check(_lib().ple_grad_scatter_noalloc(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
                                            _stream(rows.device)), "ple_grad_scatter_noalloc")
     return table_grad
+
+
+# ---------------------------------------------------------------------------
+# host-memory tier: table in pinned host memory, distinct rows prefetched
+# ---------------------------------------------------------------------------
+
+class Prefetched:
+    """Device buffers of one prefetched batch: cache [cache_rows, D], slots
+    [T, H], uniq_rows [cache_rows], num_unique (one int64 on the device)."""
+
+    def __init__(self, plan: Plan, num_tokens: int, device):
+        n = int(num_tokens) * plan.num_heads
+        self.cache_rows = max(n, 1)
+        self.cache = torch.empty(self.cache_rows, plan.head_dim, dtype=plan.table_dtype, device=device)
+        self.slots = torch.empty(int(num_tokens), plan.num_heads, dtype=torch.int64, device=device)
+        self.uniq_rows = torch.empty(self.cache_rows, dtype=torch.int64, device=device)
+        self.num_unique = torch.zeros(1, dtype=torch.int64, device=device)
+        self.workspace = torch.empty(max(int(_lib().ple_prefetch_workspace_bytes(plan.handle, int(num_tokens))), 1),
+                                     dtype=torch.uint8, device=device)
+
+
+def ple_prefetch(plan: Plan, tokens, cu_seqlens, host_table, buffers: "Prefetched" = None):
+    """Hash the batch and copy each distinct row once from host_table (a
+    pinned CPU tensor [num_rows, D] in the plan's dtype) into a device cache.
+    Runs on the current stream; returns the Prefetched buffers."""
+    _as_i64(tokens, "tokens")
+    _as_i32(cu_seqlens, "cu_seqlens")
+    if host_table.dtype != plan.table_dtype or not host_table.is_contiguous() or host_table.is_cuda \
+            or not host_table.is_pinned() or host_table.numel() != plan.num_rows * plan.head_dim:
+        raise ValueError("host_table must be a contiguous pinned CPU tensor [num_rows, head_dim] in the plan's dtype")
+    T = tokens.numel()
+    if buffers is None:
+        buffers = Prefetched(plan, T, tokens.device)
+    elif buffers.slots.numel() != T * plan.num_heads:
+        raise ValueError("buffers were made for another number of tokens")
+    _check(_lib().ple_prefetch(plan.handle, _ptr(tokens), T, _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                               host_table.data_ptr(), _ptr(buffers.cache), buffers.cache_rows, _ptr(buffers.slots),
+                               _ptr(buffers.uniq_rows), _ptr(buffers.num_unique), _ptr(buffers.workspace),
+                               buffers.workspace.numel(), _stream(tokens.device)), "ple_prefetch")
+    return buffers
+
+
+def ple_gather_cache(plan: Plan, buffers: "Prefetched", out=None):
+    """The lookup of a prefetched batch: [T, H, D] (bf16 for an fp8 table)."""
+    T, H = buffers.slots.shape
+    out = _out(plan, out, (T, H, plan.head_dim), buffers.cache.device)
+    _check(_lib().ple_gather_cache(plan.handle, _ptr(buffers.slots), T * H, _ptr(buffers.cache), buffers.cache_rows,
+                                   _ptr(out), _stream(out.device)), "ple_gather_cache")
+    return out
+
+
+def ple_grad_scatter_cache(plan: Plan, buffers: "Prefetched", grad_out, cache_grad=None, workspace=None):
+    """Deterministic gradient of a prefetched batch into cache_grad fp32
+    [cache_rows, D] (accumulated into; row u belongs to uniq_rows[u])."""
+    gdt = _grad_dtype(grad_out)
+    N = buffers.slots.numel()
+    if grad_out.numel() != N * plan.head_dim:
+        raise ValueError("grad_out must hold num_hits * head_dim values")
+    dev = buffers.cache.device
+    if cache_grad is None:
+        cache_grad = torch.zeros(buffers.cache_rows, plan.head_dim, dtype=torch.float32, device=dev)
+    elif cache_grad.dtype != torch.float32 or cache_grad.numel() != buffers.cache_rows * plan.head_dim \
+            or not cache_grad.is_contiguous():
+        raise ValueError("cache_grad must be a contiguous float32 tensor [cache_rows, head_dim]")
+    if workspace is None:
+        workspace = alloc_workspace(plan, N, dev)
+    _check(_lib().ple_grad_scatter_cache(plan.handle, _ptr(buffers.slots), N, _ptr(grad_out), gdt, _ptr(cache_grad),
+                                         buffers.cache_rows, _ptr(workspace), workspace.numel(), _stream(dev)),
+           "ple_grad_scatter_cache")
+    return cache_grad
 
 
 # ---------------------------------------------------------------------------

@@ -288,7 +288,15 @@ __global__ void conv_reduce_kernel(const float* __restrict__ part, int64_t nchun
   if (e >= n) return;
   wait_for_prior_grid();
   float sum = part[e];
-  for (int64_t q = 1; q < nchunks; ++q) sum += part[q * n + e];
+  int64_t q = 1;
+  for (; q + 8 <= nchunks; q += 8) {  // eight loads in flight, added in order
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = part[(q + u) * n + e];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sum += v[u];
+  }
+  for (; q < nchunks; ++q) sum += part[q * n + e];
   const int64_t c = e / (K + 1);
   const int k = static_cast<int>(e - c * (K + 1));
   if (k < K) {
@@ -421,7 +429,7 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
   if (e != cudaSuccess) return cuda_fail(e);
   if (want_params) {
     const int64_t n = C * (K + 1);
-    e = launch_after(conv_reduce_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s,
+    e = launch_after(conv_reduce_kernel, dim3(static_cast<unsigned>((n + 63) / 64)), dim3(64), 0, s,
                      static_cast<const float*>(part), nchunks, C, static_cast<int>(K), dweight, dbias);
     if (e != cudaSuccess) return cuda_fail(e);
   }

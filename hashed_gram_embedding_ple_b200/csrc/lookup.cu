@@ -461,6 +461,46 @@ ple_status_t dispatch_lookup(const ple_plan_t* plan, const int64_t* tokens, int6
 #undef PLE_TW_CASE
 }
 
+ple_status_t gather_bounded(const ple_plan_t* plan, const int64_t* rows, int64_t N, int64_t R, const void* table,
+                            void* out, void* stream) {
+  if (plan == nullptr || N < 0) return PLE_ERR_INVALID_ARG;
+  if (N == 0) return PLE_OK;
+  if (rows == nullptr || table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
+  if (!aligned(rows, 8) || !aligned(table, 16) || !aligned(out, 16)) return PLE_ERR_ALIGNMENT;
+  cudaError_t e;
+  unsigned int* status = status_word(&e);
+  if (status == nullptr) return cuda_fail(e);
+  const dim3 grid(static_cast<unsigned>((N + kGatherHits - 1) / kGatherHits));
+  const auto s = static_cast<cudaStream_t>(stream);
+  const auto* tb = static_cast<const unsigned char*>(table);
+  auto* ob = static_cast<unsigned char*>(out);
+  const int rb = plan->row_bytes;
+  const bool widen = plan->table_dtype == PLE_F8E4M3;
+#define PLE_GATHER_CASE(VL)                                                                   \
+  case VL:                                                                                    \
+    if (widen)                                                                                \
+      gather_kernel<VL, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);        \
+    else                                                                                      \
+      gather_kernel<VL, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);       \
+    break;
+  switch (log2_exact(rb >> 4)) {
+    PLE_GATHER_CASE(0)
+    PLE_GATHER_CASE(1)
+    PLE_GATHER_CASE(2)
+    PLE_GATHER_CASE(3)
+    PLE_GATHER_CASE(4)
+    PLE_GATHER_CASE(5)
+    PLE_GATHER_CASE(6)
+    default:
+      if (widen)
+        gather_kernel<-1, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
+      else
+        gather_kernel<-1, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
+  }
+#undef PLE_GATHER_CASE
+  return check_launch();
+}
+
 ple_status_t check_lookup_ptrs(const void* table, void* out, int64_t* rows_out) {
   if (table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(table, 16) || !aligned(out, 16) || (rows_out != nullptr && !aligned(rows_out, 8)))
@@ -497,43 +537,14 @@ ple_status_t ple_lookup_slice(const ple_plan_t* plan, const int64_t* tokens, int
 
 ple_status_t ple_gather(const ple_plan_t* plan, const int64_t* rows, int64_t N, const void* table, void* out,
                         void* stream) {
-  if (plan == nullptr || N < 0) return PLE_ERR_INVALID_ARG;
-  if (N == 0) return PLE_OK;
-  if (rows == nullptr || table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
-  if (!aligned(rows, 8) || !aligned(table, 16) || !aligned(out, 16)) return PLE_ERR_ALIGNMENT;
-  cudaError_t e;
-  unsigned int* status = status_word(&e);
-  if (status == nullptr) return cuda_fail(e);
-  const dim3 grid(static_cast<unsigned>((N + kGatherHits - 1) / kGatherHits));
-  const auto s = static_cast<cudaStream_t>(stream);
-  const auto* tb = static_cast<const unsigned char*>(table);
-  auto* ob = static_cast<unsigned char*>(out);
-  const int rb = plan->row_bytes;
-  const int64_t R = plan->num_rows;
-  const bool widen = plan->table_dtype == PLE_F8E4M3;
-#define PLE_GATHER_CASE(VL)                                                                   \
-  case VL:                                                                                    \
-    if (widen)                                                                                \
-      gather_kernel<VL, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);        \
-    else                                                                                      \
-      gather_kernel<VL, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);       \
-    break;
-  switch (log2_exact(rb >> 4)) {
-    PLE_GATHER_CASE(0)
-    PLE_GATHER_CASE(1)
-    PLE_GATHER_CASE(2)
-    PLE_GATHER_CASE(3)
-    PLE_GATHER_CASE(4)
-    PLE_GATHER_CASE(5)
-    PLE_GATHER_CASE(6)
-    default:
-      if (widen)
-        gather_kernel<-1, true><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
-      else
-        gather_kernel<-1, false><<<grid, kBlock, 0, s>>>(rows, N, R, tb, rb, ob, status);
-  }
-#undef PLE_GATHER_CASE
-  return check_launch();
+  if (plan == nullptr) return PLE_ERR_INVALID_ARG;
+  return gather_bounded(plan, rows, N, plan->num_rows, table, out, stream);
+}
+
+ple_status_t ple_gather_cache(const ple_plan_t* plan, const int64_t* slots, int64_t N, const void* cache,
+                              int64_t cache_rows, void* out, void* stream) {
+  if (plan == nullptr || cache_rows < 0) return PLE_ERR_INVALID_ARG;
+  return gather_bounded(plan, slots, N, cache_rows, cache, out, stream);
 }
 
 }  // extern "C"

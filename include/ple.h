@@ -191,6 +191,52 @@ ple_status_t ple_grad_scatter_noalloc(const ple_plan_t* plan, const int64_t* row
 /* Bytes of the fixed scratch area ple_grad_scatter_noalloc works in. */
 size_t ple_grad_scatter_noalloc_scratch_bytes(void);
 
+/* ---- Host-memory tier ----------------------------------------------------------
+ * The table stays in pinned host memory and the rows a batch touches are
+ * brought to the GPU ahead of its lookup: the CPU offload of the n-gram table
+ * with asynchronous prefetch ("add native Qwen3.8 Flash Next" pull request,
+ * Summary and Overview: ngram_embedding_cpu_offload).
+ *
+ * ple_prefetch hashes the batch exactly as ple_hash, then, for the distinct
+ * rows of its num_tokens * H hits in ascending order:
+ *   uniq_rows[u] = the u-th distinct row (-1 for a row outside the table),
+ *   cache[u, :] = host_table[uniq_rows[u], :] (raw copy in the table dtype),
+ *   slots[t*H + j] = u for every hit of that row, *num_unique = the count.
+ * Every distinct row is read once over the host link, with 16-byte loads
+ * from the mapped host memory.  host_table: [num_rows, head_dim] in host
+ * memory the device can read (pinned: cudaHostAlloc / cudaHostRegister on a
+ * system with unified addressing; device or managed memory also works);
+ * pageable memory is rejected with PLE_ERR_INVALID_ARG.  cache [cache_rows,
+ * head_dim] table dtype and uniq_rows int64 [cache_rows] on the device,
+ * cache_rows >= num_tokens * H (room for every hit); slots int64
+ * [num_tokens, H]; num_unique: one int64 in device memory.  host_table and
+ * cache 16-byte aligned, workspace (ple_prefetch_workspace_bytes) 256-byte
+ * aligned.  Run it on a side stream for the next batch to overlap the copy
+ * with the current batch's compute.  num_tokens == 0 writes *num_unique = 0.
+ * Errors as ple_hash, plus PLE_ERR_WORKSPACE, PLE_ERR_ALIGNMENT,
+ * PLE_ERR_UNSUPPORTED (num_tokens * H >= 2^31). */
+size_t ple_prefetch_workspace_bytes(const ple_plan_t* plan, int64_t num_tokens);
+ple_status_t ple_prefetch(const ple_plan_t* plan, const int64_t* tokens, int64_t num_tokens, const int32_t* cu_seqlens,
+                          int32_t num_seqs, const void* host_table, void* cache, int64_t cache_rows, int64_t* slots,
+                          int64_t* uniq_rows, int64_t* num_unique, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* The lookup of a prefetched batch: out[i, :] = cache[slots[i], :] (bf16 for
+ * an E4M3 table), as ple_gather with the cache for the table; a slot outside
+ * [0, cache_rows) yields a zero row and the async PLE_ERR_BAD_ROW. */
+ple_status_t ple_gather_cache(const ple_plan_t* plan, const int64_t* slots, int64_t num_hits, const void* cache,
+                              int64_t cache_rows, void* out, void* stream);
+
+/* The backward of a prefetched batch: the deterministic gradient of
+ * ple_grad_scatter with the slots for rows, summed into cache_grad fp32
+ * [cache_rows, head_dim] (accumulated into); row u of cache_grad is the
+ * gradient of table row uniq_rows[u], to be applied on the host.  Same
+ * summation order, workspace (ple_grad_scatter_workspace_bytes) and errors as
+ * ple_grad_scatter, with cache_rows as the row bound. */
+ple_status_t ple_grad_scatter_cache(const ple_plan_t* plan, const int64_t* slots, int64_t num_hits, const void* grad_out,
+                                    ple_dtype_t grad_dtype, float* cache_grad, int64_t cache_rows, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* ---- The PLE layer's short convolution --------------------------------------
  * Segment-aware causal dilated depthwise convolution over packed tokens
  * (Qwen3_8_FlashNextPLELayer._causal_short_conv and _segmented_conv, NeMo

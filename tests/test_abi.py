@@ -162,3 +162,31 @@ def test_conv_rejects_bad_arguments_on_host():
         binding.PLE_ERR_ALIGNMENT
     # 1024 chunks at most: the workspace stops growing with the token count past 256 K tokens
     assert lib.ple_conv_backward_workspace_bytes(1 << 24, 8, 4) == 1024 * 8 * 5 * 4
+
+
+def test_host_tier_rejects_bad_arguments_on_host():
+    lib = ple.lib()
+    p = _plan()  # 4 heads
+    h = p.handle
+    pf = lib.ple_prefetch
+    # empty: only the device count is written -> needs a count pointer
+    assert pf(h, None, 0, None, 0, None, None, 0, None, None, None, None, 0, None) == binding.PLE_ERR_INVALID_ARG
+    # null pointers; a cache smaller than the hits (5 tokens x 4 heads = 20)
+    assert pf(h, None, 5, 0x2000, 1, 0x3000, 0x4000, 20, 0x5000, 0x6000, 0x7000, 0x8000, 1 << 20, None) == \
+        binding.PLE_ERR_INVALID_ARG
+    assert pf(h, 0x1000, 5, 0x2000, 1, 0x3000, 0x4000, 19, 0x5000, 0x6000, 0x7000, 0x8000, 1 << 20, None) == \
+        binding.PLE_ERR_INVALID_ARG
+    # misaligned host table / cache / slots
+    assert pf(h, 0x1000, 5, 0x2000, 1, 0x3008, 0x4000, 20, 0x5000, 0x6000, 0x7000, 0x8000, 1 << 20, None) == \
+        binding.PLE_ERR_ALIGNMENT
+    assert pf(h, 0x1000, 5, 0x2000, 1, 0x3000, 0x4008, 20, 0x5000, 0x6000, 0x7000, 0x8000, 1 << 20, None) == \
+        binding.PLE_ERR_ALIGNMENT
+    assert pf(h, 0x1000, 5, 0x2000, 1, 0x3000, 0x4000, 20, 0x5004, 0x6000, 0x7000, 0x8000, 1 << 20, None) == \
+        binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_prefetch_workspace_bytes(h, 5) > 0 and lib.ple_prefetch_workspace_bytes(h, 0) == 0
+    # gather and gradient from a cache: the usual checks, the cache size as the bound
+    assert lib.ple_gather_cache(h, None, 0, None, 10, None, None) == 0
+    assert lib.ple_gather_cache(h, 0x1000, 5, 0x2000, -1, 0x3000, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_gather_cache(h, 0x1000, 5, 0x2008, 10, 0x3000, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_grad_scatter_cache(h, 0x1000, 5, 0x2000, 1, 0x3000, 0, 0x4000, 1 << 20, None) == \
+        binding.PLE_ERR_INVALID_ARG
