@@ -239,6 +239,9 @@ def main():
     ap.add_argument("--conv", action="store_true",
                     help="time the PLE layer's short convolution (forward + backward) instead of the lookup")
     ap.add_argument("--conv-channels", type=int, default=8192, help="channels of the --conv workload")
+    ap.add_argument("--host-table", action="store_true",
+                    help="keep the table in pinned host memory: time ple_prefetch, the cached lookup and gradient, "
+                         "and the two-stream pipeline")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -270,6 +273,8 @@ def main():
 
     if args.conv:
         return run_conv(args, rank, world, dev, dist)
+    if args.host_table:
+        return run_host_table(args, rank, world, dev, dist)
     w = workload(args.workload, replica_seed(args.seed, rank))
     plan = ple.Plan.from_workload(w)
     T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
@@ -625,6 +630,147 @@ def run_conv(args, rank, world, dev, dist):
                         "frac_of_measured": bwd_gbs / peak},
                 "roofline": roofline, "roofline_fwd": roof_f, "roofline_bwd": roof_b, "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks, "wall_s_timed_region": wall}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_host_table(args, rank, world, dev, dist):
+    """--host-table: the workload's table in pinned host memory.  Times, with
+    CUDA events: ple_prefetch (the distinct rows over the host link), the
+    cached lookup, the cached gradient, and a two-stream pipeline in which the
+    prefetch of batch k+1 runs beside the lookup + gradient of batch k (two
+    buffer sets, events between the streams).  The link's own peak is a
+    pinned host-to-device copy of 256 MB measured in the same run."""
+    import torch
+
+    import hashed_gram_embedding_ple_b200 as ple
+    from synth import gpu as sgpu
+
+    w = workload(args.workload, replica_seed(args.seed, rank))
+    plan = ple.Plan.from_workload(w)
+    T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
+    tdt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float8_e4m3fn}[w.table_dtype]
+    dtab = torch.empty(w.num_rows, D, dtype=tdt, device=dev)
+    sgpu.fill_(dtab, w.table_seed, w.table_sigma)
+    table = torch.empty(w.num_rows, D, dtype=tdt, pin_memory=True)
+    table.copy_(dtab)
+    del dtab
+    tokens = torch.from_numpy(w.tokens).to(dev)
+    cu = torch.from_numpy(w.cu_seqlens).to(dev)
+    grad = torch.empty(N, D, dtype=torch.bfloat16 if w.grad_dtype == 1 else torch.float32, device=dev)
+    sgpu.fill_(grad, w.grad_seed, w.grad_sigma)
+    bufs = [ple.Prefetched(plan, T, dev) for _ in range(2)]
+    outs = [torch.empty(T, H, D, dtype=plan.out_dtype, device=dev) for _ in range(2)]
+    cgrads = [torch.zeros(b.cache_rows, D, dtype=torch.float32, device=dev) for b in bufs]
+    ws = ple.alloc_workspace(plan, N, dev)
+    main = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush_w.zero_()
+        flush_r.sum()
+
+    def compute(i):
+        ple.ple_gather_cache(plan, bufs[i], out=outs[i])
+        ple.ple_grad_scatter_cache(plan, bufs[i], grad, cache_grad=cgrads[i], workspace=ws)
+
+    # link peak: pinned host -> device copy
+    h = torch.empty(256 << 20, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        d.copy_(h, non_blocking=True)
+    e0.record(main)
+    for _ in range(4):
+        d.copy_(h, non_blocking=True)
+    e1.record(main)
+    torch.cuda.synchronize()
+    link_gbs = 4 * h.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del h, d
+
+    for _ in range(args.warmup):
+        flush_l2()
+        ple.ple_prefetch(plan, tokens, cu, table, bufs[0])
+        compute(0)
+    torch.cuda.synchronize()
+    if ple.ple_status(dev) != ple.PLE_OK:
+        raise SystemExit("libple async status after warm-up")
+    U = int(bufs[0].num_unique.item())
+    # each part alone
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush_l2()
+        ev[k][0].record(main)
+        ple.ple_prefetch(plan, tokens, cu, table, bufs[0])
+        ev[k][1].record(main)
+        ple.ple_gather_cache(plan, bufs[0], out=outs[0])
+        ev[k][2].record(main)
+        ple.ple_grad_scatter_cache(plan, bufs[0], grad, cache_grad=cgrads[0], workspace=ws)
+        ev[k][3].record(main)
+    torch.cuda.synchronize()
+    ms_pf = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps))
+    ms_lk = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps))
+    ms_bw = statistics.mean(ev[k][2].elapsed_time(ev[k][3]) for k in range(args.steps))
+    # pipeline: prefetch of batch k+1 on the side stream beside batch k's compute
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
+    with torch.cuda.stream(side):
+        ple.ple_prefetch(plan, tokens, cu, table, bufs[0])
+        ready[0].record(side)
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.perf_counter()
+    p0.record(main)
+    for k in range(args.steps):
+        i, j = k % 2, (k + 1) % 2
+        with torch.cuda.stream(side):  # the next batch (the same tokens, a new prefetch)
+            if k > 0:
+                side.wait_event(free[j])
+            ple.ple_prefetch(plan, tokens, cu, table, bufs[j])
+            ready[j].record(side)
+        main.wait_event(ready[i])
+        compute(i)
+        free[i].record(main)
+    p1.record(main)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    if ple.ple_status(dev) != ple.PLE_OK:
+        raise SystemExit("libple async status after the pipeline")
+    (ms_pipe,) = reduce_max([p0.elapsed_time(p1) / args.steps], dist, dev)
+    ms_pf, ms_lk, ms_bw = reduce_max([ms_pf, ms_lk, ms_bw], dist, dev)
+    pf_bytes = U * plan.table_dtype.itemsize * D  # the distinct rows over the link
+    e_o = outs[0].element_size()
+    lk_bytes = N * (8 + plan.table_dtype.itemsize * D + e_o * D)
+    pf_gbs = pf_bytes / (ms_pf * 1e-3) / 1e9
+    roof = {"bound": "pcie", "achieved": pf_gbs, "peak": link_gbs, "unit": "GB/s", "frac": pf_gbs / link_gbs,
+            "algorithmic_bytes": pf_bytes, "traffic": None, "kernel": "ple_prefetch (finalize_kernel row copies)",
+            "peak_source": "measured in this run: pinned host-to-device copy of 256 MB"}
+    if rank == 0:
+        line = {"metric": "PLE lookup tokens/s with the table in pinned host memory (prefetch pipelined)",
+                "value": world * T / (ms_pipe * 1e-3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_pipe, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": f"int64 hash, {DTYPE_NAMES[w.table_dtype]} rows over the host link",
+                "data": "synthetic",
+                "config": dict(describe(w), parallelism=f"replicas{world}", table_location="pinned host memory",
+                               unique_rows=U,
+                               step="ple_prefetch of the next batch (side stream) beside ple_gather_cache + "
+                                    "ple_grad_scatter_cache of the current one"),
+                "parts_ms": {"prefetch": ms_pf, "gather_cache": ms_lk, "grad_scatter_cache": ms_bw},
+                "prefetch_gb_per_s": pf_gbs, "link_peak_gb_per_s": link_gbs,
+                "gather_cache_gb_per_s": lk_bytes / (ms_lk * 1e-3) / 1e9,
+                "roofline": roof, "cpu_baseline": None, "e2e": None,
+                "gpu_launches": None, "clocks": clocks, "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
