@@ -43,6 +43,12 @@ __device__ __forceinline__ void order_hashes(const HashParams& hp, const int64_t
                                              bool valid, int64_t (&hs)[kMaxOrder - 1]) {
   const int lane = threadIdx.x & 31;
   const int64_t tok = valid ? tokens[t] : 0;
+  // the halo (tokens before the warp's first) is loaded together with the
+  // lane's own token, ahead of the segment search: one round trip, not two
+  int64_t halo[kMaxOrder];
+#pragma unroll
+  for (int k = 1; k < kMaxOrder; ++k)
+    halo[k] = (k < hp.ngram_size && lane < k && valid && t - k >= 0) ? tokens[t - k] : 0;
   const int64_t seq_start = valid ? static_cast<int64_t>(cu[find_sequence(cu, num_seqs, t)]) : 0;
   uint64_t h = static_cast<uint64_t>(tok) * static_cast<uint64_t>(hp.mults[0]);
   bool keep = valid;
@@ -50,7 +56,7 @@ __device__ __forceinline__ void order_hashes(const HashParams& hp, const int64_t
   for (int k = 1; k < kMaxOrder; ++k) {
     if (k < hp.ngram_size) {
       int64_t prev = __shfl_up_sync(kFull, tok, k);
-      if (lane < k) prev = (valid && t - k >= 0) ? tokens[t - k] : 0;
+      if (lane < k) prev = halo[k];
       keep = keep && (t - k >= seq_start) && (prev != hp.eos_id);
       const int64_t ctx = keep ? prev : 0;
       h += static_cast<uint64_t>(ctx) * static_cast<uint64_t>(hp.mults[k]);
