@@ -36,7 +36,8 @@ _DTYPE_OF_CODE = {PLE_F32: torch.float32, PLE_BF16: torch.bfloat16, PLE_F8E4M3: 
 # every symbol include/ple.h declares
 EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_hash", "ple_lookup", "ple_lookup_slice",
            "ple_gather",
-           "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_scatter_atomic",
+           "ple_grad_scatter_workspace_bytes", "ple_grad_scatter", "ple_grad_prepare", "ple_grad_apply",
+           "ple_grad_scatter_atomic",
            "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_prefetch_workspace_bytes",
            "ple_prefetch", "ple_gather_cache", "ple_grad_scatter_cache", "ple_conv_forward",
            "ple_conv_backward_workspace_bytes", "ple_conv_backward", "ple_status", "ple_strerror",
@@ -82,6 +83,8 @@ def _lib():
         lib.ple_grad_scatter_workspace_bytes.argtypes = [vp, i64]
         lib.ple_grad_scatter_workspace_bytes.restype = sz
         lib.ple_grad_scatter.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
+        lib.ple_grad_prepare.argtypes = [vp, vp, i64, vp, sz, vp]
+        lib.ple_grad_apply.argtypes = [vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]
         lib.ple_grad_scatter_atomic.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
         lib.ple_grad_scatter_noalloc.argtypes = [vp, vp, i64, vp, ctypes.c_int, vp, vp]
         lib.ple_grad_scatter_noalloc_scratch_bytes.argtypes = []
@@ -101,6 +104,7 @@ def _lib():
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
         for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_lookup_slice", "ple_gather", "ple_grad_scatter",
+                     "ple_grad_prepare", "ple_grad_apply",
                      "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_prefetch", "ple_gather_cache",
                      "ple_grad_scatter_cache", "ple_conv_forward",
                      "ple_conv_backward", "ple_status", "ple_last_cuda_error"):
@@ -301,6 +305,27 @@ def ple_grad_scatter(plan: Plan, rows, grad_out, table_grad, workspace=None):
         workspace = alloc_workspace(plan, N, rows.device)
     _check(_lib().ple_grad_scatter(plan.handle, _ptr(rows), N, _ptr(grad_out), gdt, _ptr(table_grad),
                                    _ptr(workspace), workspace.numel(), _stream(rows.device)), "ple_grad_scatter")
+    return table_grad
+
+
+def ple_grad_prepare(plan: Plan, rows, workspace):
+    """First half of ple_grad_scatter: sort the rows into the workspace (it
+    must then stay untouched until the matching ple_grad_apply)."""
+    _as_i64(rows, "rows")
+    N = rows.numel()
+    _check(_lib().ple_grad_prepare(plan.handle, _ptr(rows), N, _ptr(workspace), workspace.numel(),
+                                   _stream(rows.device)), "ple_grad_prepare")
+    return workspace
+
+
+def ple_grad_apply(plan: Plan, num_hits: int, grad_out, table_grad, workspace):
+    """Second half: fold grad_out in the prepared order into table_grad."""
+    gdt = _grad_dtype(grad_out)
+    _check_table_grad(plan, table_grad)
+    if grad_out.numel() != int(num_hits) * plan.head_dim:
+        raise ValueError("grad_out must hold num_hits * head_dim values")
+    _check(_lib().ple_grad_apply(plan.handle, int(num_hits), _ptr(grad_out), gdt, _ptr(table_grad), _ptr(workspace),
+                                 workspace.numel(), _stream(grad_out.device)), "ple_grad_apply")
     return table_grad
 
 

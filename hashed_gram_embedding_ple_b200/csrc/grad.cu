@@ -681,12 +681,24 @@ namespace {
 
 // The deterministic gradient with an explicit row bound: rows in
 // [0, num_rows) are summed into table_grad [num_rows, head_dim], others are
-// dropped (and flagged).
+// dropped (and flagged).  The phases: kPrepare sorts the rows into the
+// workspace (it does not read grad_out); kApply folds grad_out in the
+// sorted order (it does not read the rows); kBoth does both in order.
+enum Phase { kPrepare = 1, kApply = 2, kBoth = 3 };
+
 ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, int64_t N, int64_t num_rows,
                                   const void* grad, ple_dtype_t gdt, float* table_grad, void* workspace,
-                                  size_t ws_bytes, void* stream) {
-  ple_status_t st = check_grad_args(plan, rows, N, grad, gdt, table_grad);
-  if (st != PLE_OK || N == 0) return st;
+                                  size_t ws_bytes, void* stream, int phases = kBoth) {
+  if (plan == nullptr || N < 0) return PLE_ERR_INVALID_ARG;
+  if ((phases & kApply) && gdt != PLE_F32 && gdt != PLE_BF16) return PLE_ERR_INVALID_ARG;
+  if (N == 0) return PLE_OK;
+  if ((phases & kPrepare) && rows == nullptr) return PLE_ERR_INVALID_ARG;
+  if ((phases & kApply) && (grad == nullptr || table_grad == nullptr)) return PLE_ERR_INVALID_ARG;
+  if (plan->head_dim > 32 * kMaxColsPerLane) return PLE_ERR_UNSUPPORTED;
+  if ((phases & kPrepare) && !aligned(rows, 8)) return PLE_ERR_ALIGNMENT;
+  if ((phases & kApply) && (!aligned(grad, 16) || !aligned(table_grad, 16) ||
+                            (static_cast<int64_t>(plan->head_dim) * (gdt == PLE_F32 ? 4 : 2)) % 16 != 0))
+    return PLE_ERR_ALIGNMENT;
   if (num_rows < 1) return PLE_ERR_INVALID_ARG;
   if (num_rows >= static_cast<int64_t>(kNoKey) || N >= (int64_t{1} << 31)) return PLE_ERR_UNSUPPORTED;
   const int D = plan->head_dim;
@@ -704,8 +716,13 @@ ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, i
   rb.done = reinterpret_cast<unsigned int*>(ws + L.run_done);
   const uint32_t* Ks = nullptr;
   const uint32_t* Is = nullptr;
-  st = launch_sort(rows, N, num_rows, ws, L.sort, rb.done, L.nwin, status, s, &Ks, &Is);
-  if (st != PLE_OK) return st;
+  if (phases & kPrepare) {
+    ple_status_t st = launch_sort(rows, N, num_rows, ws, L.sort, rb.done, L.nwin, status, s, &Ks, &Is);
+    if (st != PLE_OK) return st;
+    if (!(phases & kApply)) return check_launch();
+  } else {
+    sorted_result(L.sort, num_rows, ws, &Ks, &Is);
+  }
   const uint32_t bad_key = static_cast<uint32_t>(num_rows);
   const dim3 fold_grid(static_cast<unsigned>((L.nwin * 32 + kFoldThreads - 1) / kFoldThreads));
   const bool bf = gdt == PLE_BF16;
@@ -740,6 +757,20 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
                               void* stream) {
   if (plan == nullptr) return PLE_ERR_INVALID_ARG;
   return grad_scatter_bounded(plan, rows, N, plan->num_rows, grad, gdt, table_grad, workspace, ws_bytes, stream);
+}
+
+ple_status_t ple_grad_prepare(const ple_plan_t* plan, const int64_t* rows, int64_t N, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (plan == nullptr) return PLE_ERR_INVALID_ARG;
+  return grad_scatter_bounded(plan, rows, N, plan->num_rows, nullptr, PLE_F32, nullptr, workspace, ws_bytes, stream,
+                              kPrepare);
+}
+
+ple_status_t ple_grad_apply(const ple_plan_t* plan, int64_t N, const void* grad, ple_dtype_t gdt, float* table_grad,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  if (plan == nullptr) return PLE_ERR_INVALID_ARG;
+  return grad_scatter_bounded(plan, nullptr, N, plan->num_rows, grad, gdt, table_grad, workspace, ws_bytes, stream,
+                              kApply);
 }
 
 ple_status_t ple_grad_scatter_cache(const ple_plan_t* plan, const int64_t* slots, int64_t N, const void* grad,

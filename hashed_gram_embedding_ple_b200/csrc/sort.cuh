@@ -372,6 +372,21 @@ inline SortLayout sort_layout(int64_t N, size_t* off) {
   return L;
 }
 
+// 8-bit digit passes for keys in [0, num_rows] (num_rows marks a bad row).
+inline int sort_passes(int64_t num_rows) {
+  int bits = 0;
+  while (bits < 32 && (static_cast<uint64_t>(num_rows) >> bits) != 0) ++bits;
+  return (bits + 7) / 8 > 1 ? (bits + 7) / 8 : 1;
+}
+
+// Where the sort leaves its result (keys, values) for keys below num_rows.
+inline void sorted_result(const SortLayout& L, int64_t num_rows, unsigned char* ws, const uint32_t** keys,
+                          const uint32_t** vals) {
+  const int b = sort_passes(num_rows) & 1;
+  *keys = reinterpret_cast<const uint32_t*>(ws + L.keys[b]);
+  *vals = reinterpret_cast<const uint32_t*>(ws + L.vals[b]);
+}
+
 // Sorts the N rows (keys in [0, num_rows]; a row outside [0, num_rows)
 // becomes the key num_rows) with their hit indices: clear, key_hist, one pass
 // per 8-bit digit, all launched with programmatic dependent launch.  On
@@ -393,9 +408,7 @@ inline ple_status_t launch_sort(const int64_t* rows, int64_t N, int64_t num_rows
   sa.hist = reinterpret_cast<uint32_t*>(ws + L.zeroed);
   sa.tickets = sa.hist + kMaxPasses * kRadix;
   sa.status = status;
-  int bits = 0;  // key bits: keys lie in [0, num_rows]
-  while (bits < 32 && (static_cast<uint64_t>(num_rows) >> bits) != 0) ++bits;
-  sa.passes = (bits + 7) / 8 > 1 ? (bits + 7) / 8 : 1;
+  sa.passes = sort_passes(num_rows);
   cudaError_t e = launch_after(clear_kernel, dim3(1), dim3(kSortThreads), 0, s, sa.hist,
                                static_cast<int>(L.zeroed_bytes / sizeof(uint32_t)));
   if (e != cudaSuccess) return cuda_fail(e);

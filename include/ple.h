@@ -161,6 +161,22 @@ ple_status_t ple_grad_scatter(const ple_plan_t* plan, const int64_t* rows, int64
                               const void* grad_out, ple_dtype_t grad_dtype, float* table_grad,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ple_grad_scatter in two halves, for callers that want the row sort out of
+ * the backward's critical path.  The sort depends only on the rows, not on
+ * grad_out, so ple_grad_prepare can run as soon as the rows exist (for
+ * instance on a second stream beside the forward gather, hashing the tokens
+ * with ple_hash), and ple_grad_apply later folds grad_out in the prepared
+ * order.  Together they compute exactly ple_grad_scatter (same order, same
+ * bits).  The workspace (ple_grad_scatter_workspace_bytes for num_hits)
+ * carries the prepared state: leave it untouched between the two calls, pass
+ * the same plan and num_hits, and use one prepare for one apply (the apply
+ * consumes counters the prepare cleared).  Errors as ple_grad_scatter, each
+ * call checking its own arguments. */
+ple_status_t ple_grad_prepare(const ple_plan_t* plan, const int64_t* rows, int64_t num_hits, void* workspace,
+                              size_t workspace_bytes, void* stream);
+ple_status_t ple_grad_apply(const ple_plan_t* plan, int64_t num_hits, const void* grad_out, ple_dtype_t grad_dtype,
+                            float* table_grad, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Same sums by fp32 atomic adds, one per hit and column: no workspace and
  * no fixed order (results can differ in the last bits run to run).  A speed
  * reference for the deterministic path; same argument rules. */

@@ -190,3 +190,18 @@ def test_host_tier_rejects_bad_arguments_on_host():
     assert lib.ple_gather_cache(h, 0x1000, 5, 0x2008, 10, 0x3000, None) == binding.PLE_ERR_ALIGNMENT
     assert lib.ple_grad_scatter_cache(h, 0x1000, 5, 0x2000, 1, 0x3000, 0, 0x4000, 1 << 20, None) == \
         binding.PLE_ERR_INVALID_ARG
+
+
+def test_grad_halves_check_their_own_arguments():
+    lib = ple.lib()
+    p = _plan()
+    h = p.handle
+    need = lib.ple_grad_scatter_workspace_bytes(h, 5)
+    assert lib.ple_grad_prepare(h, None, 0, None, 0, None) == 0
+    assert lib.ple_grad_prepare(h, None, 5, 0x4000, need, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_grad_prepare(h, 0x1004, 5, 0x4000, need, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_grad_prepare(h, 0x1000, 5, 0x4000, need - 1, None) == binding.PLE_ERR_WORKSPACE
+    assert lib.ple_grad_apply(h, 5, None, 1, 0x3000, 0x4000, need, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_grad_apply(h, 5, 0x2000, 9, 0x3000, 0x4000, need, None) == binding.PLE_ERR_INVALID_ARG
+    assert lib.ple_grad_apply(h, 5, 0x2008, 1, 0x3000, 0x4000, need, None) == binding.PLE_ERR_ALIGNMENT
+    assert lib.ple_grad_apply(h, 5, 0x2000, 1, 0x3000, 0x4100, need - 256, None) == binding.PLE_ERR_WORKSPACE

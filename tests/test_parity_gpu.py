@@ -241,3 +241,33 @@ def test_global_slice_lookup(cuda_device, row_len, B, start, end):
     assert out.shape == (B, end - start, w.num_heads, w.head_dim)
     np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)
     np.testing.assert_array_equal(torch_to_values(out), ref_vals)
+
+
+def test_prepare_then_apply_equals_scatter(cuda_device):
+    """The two halves of the gradient, the prepare on a second stream beside
+    other work, give the same bits as ple_grad_scatter."""
+    dev = cuda_device
+    rng = np.random.default_rng(21)
+    lens = [3, 700, 0, 4000, 1]
+    tok = rng.integers(0, 40, sum(lens))  # heavy repeats: long runs
+    w = custom_workload("split", tok, synth.cu_seqlens_from_lengths(lens), 3, 4, 0, synth.signed_mults(3, rng),
+                        synth.consecutive_primes(97, 8), 64, synth.DTYPE_BF16, synth.DTYPE_BF16, seed=4)
+    plan = ple.Plan.from_workload(w)
+    tok_d, cu_d = dev_i64(w.tokens, dev), dev_i32(w.cu_seqlens, dev)
+    g = values_to_torch(host_grad(w), w.grad_dtype).to(dev)
+    N = w.num_hits
+    ref = torch.zeros(w.num_rows, w.head_dim, device=dev)
+    ple.ple_grad_scatter(plan, ple.ple_hash(plan, tok_d, cu_d).view(-1), g, ref)
+    side = torch.cuda.Stream(dev)
+    ws = ple.alloc_workspace(plan, N, dev)
+    with torch.cuda.stream(side):
+        rows = ple.ple_hash(plan, tok_d, cu_d)
+        ple.ple_grad_prepare(plan, rows.view(-1), ws)
+    _, table = small_table(w, dev)
+    out = ple.ple_lookup(plan, tok_d, cu_d, table)  # the forward, concurrently on the main stream
+    torch.cuda.current_stream(dev).wait_stream(side)
+    tg = torch.zeros(w.num_rows, w.head_dim, device=dev)
+    ple.ple_grad_apply(plan, N, g, tg, ws)
+    assert ple.ple_status() == ple.PLE_OK
+    assert out.shape == (w.num_tokens, w.num_heads, w.head_dim)
+    assert torch.equal(tg.view(torch.int32), ref.view(torch.int32))
