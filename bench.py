@@ -380,7 +380,8 @@ def main():
 
     # roofline of the dominant call of the step
     lookup_src = ["hashed_gram_embedding_ple_b200/csrc/lookup.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
-    grad_src = ["hashed_gram_embedding_ple_b200/csrc/grad.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+    grad_src = ["hashed_gram_embedding_ple_b200/csrc/grad.cu", "hashed_gram_embedding_ple_b200/csrc/sort.cuh",
+                "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
     fwd_roof = {"bound": "hbm", "achieved": fwd_gbs, "peak": peak, "unit": "GB/s", "frac": fwd_gbs / peak,
                 "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": fwd_bytes,
                 "traffic": traffic_from_profiles(f"lookup_{w.name}", lookup_src), "kernel": "lookup_kernel",
