@@ -12,9 +12,10 @@
 // load and store of a warp covers 512 consecutive bytes of a token row and
 // each row is loaded once (plus K-1 rows of history per class and chunk).
 // The backward pass computes dx (the same taps looking ahead, inside the
-// segment) and, in the same sweep, per-chunk partial sums of dw and db; a
-// second kernel adds the chunk partials in chunk order (deterministic) and
-// adds the result once into the caller's dw and db.
+// segment) in one kernel and per-chunk partial sums of dw and db in another
+// (dy is read by both; apart, each keeps few enough registers to have its
+// rows in flight); a third kernel adds the chunk partials in chunk order
+// (deterministic) and adds the result once into the caller's dw and db.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -27,6 +28,13 @@ constexpr int kConvChunk = 128;       // tokens per block, forward
 constexpr int kConvBwdChunk = 256;    // least tokens per block, backward
 constexpr int64_t kMaxPartials = 1024;  // at most this many backward chunks (their partial sums)
 constexpr int kMaxTaps = 8;
+
+// Blocks per SM the register budget is cut for (measured: more rows in
+// flight beats fewer, until the row registers start to spill); larger K
+// holds more rows and gets fewer blocks.
+constexpr int fwd_min_blocks(int K) { return K <= 4 ? 5 : K <= 5 ? 4 : K <= 7 ? 3 : 2; }
+constexpr int dx_min_blocks(int K) { return K <= 4 ? 4 : K <= 7 ? 3 : 2; }
+constexpr int dw_min_blocks(int K) { return K <= 4 ? 4 : K <= 5 ? 3 : 2; }
 
 template <bool BF16>
 struct Vec {
@@ -113,7 +121,7 @@ __device__ void check_cu(const int32_t* __restrict__ cu, int32_t num_seqs, int64
 // per output, K of them in flight; the K-1 rows before the chunk come from
 // one load each at the start of every chain.
 template <bool BF16, int K>
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, fwd_min_blocks(K))
 conv_forward_kernel(const unsigned char* __restrict__ x, int64_t T, int64_t nvec, const int32_t* __restrict__ cu,
                     int32_t num_seqs, const float* __restrict__ w, int dilation,
                     const float* __restrict__ bias, unsigned char* __restrict__ y, unsigned int* status) {
@@ -134,22 +142,23 @@ conv_forward_kernel(const unsigned char* __restrict__ x, int64_t T, int64_t nvec
   const unsigned char* xc = x + cv * 16;
   unsigned char* yc = y + cv * 16;
   Segment sg{cu, num_seqs, 0, T, 0, 0};
+  constexpr int U = 2 * K;  // chain steps per iteration: U row loads in flight
   for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
     sg.start(t0 + r);
-    uint4 prev[K], cur[K];  // chain rows: prev = the K steps before cur
+    uint4 prev[K], cur[U];  // chain rows: prev = the K steps before cur
 #pragma unroll
     for (int j = 1; j < K; ++j) {  // steps -1 .. -(K-1) before the chain's first token
       const int64_t t = t0 + r - static_cast<int64_t>(K - j) * d;
       prev[j] = t >= 0 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
     }
-    for (int64_t tb = t0 + r; tb < t1; tb += K * d) {
+    for (int64_t tb = t0 + r; tb < t1; tb += U * d) {
 #pragma unroll
-      for (int m = 0; m < K; ++m) {
+      for (int m = 0; m < U; ++m) {
         const int64_t t = tb + m * d;
         cur[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int m = 0; m < K; ++m) {
+      for (int m = 0; m < U; ++m) {
         const int64_t t = tb + m * d;
         if (t < t1) {
           sg.advance(t);
@@ -171,112 +180,158 @@ conv_forward_kernel(const unsigned char* __restrict__ x, int64_t T, int64_t nvec
         }
       }
 #pragma unroll
-      for (int m = 0; m < K; ++m) prev[m] = cur[m];
+      for (int m = 0; m < K; ++m) prev[m] = cur[U - K + m];
     }
   }
 }
 
-// Backward sweep: dx (nullable) and this chunk's partial sums of dw and db,
-// written to part[chunk][c][K + 1] (tap k at k, the bias at K).  The same
-// residue chains as the forward: output t took x at chain steps 0..K-1 back
-// (dw), and x[t] fed the outputs at chain steps 0..K-1 ahead (dx).  Per K
-// chain steps a thread loads K rows of x (the current steps) and K rows of
-// dy (K steps ahead); the rest comes from the previous iteration's registers.
+// dx of the backward: dx[t] = sum_k w[k] * dy[t + d (K-1-k)] over the taps
+// that stay inside t's segment, the forward's structure mirrored: residue
+// chains of the chunk, 2K chain steps per iteration.  Each iteration loads
+// the dy rows of the next one while it computes from the rows the iteration
+// before loaded (and the first K-1 of its own loads), so a thread always has
+// a full iteration of rows in flight.
 template <bool BF16, int K>
-__global__ void __launch_bounds__(kConvThreads)
-conv_backward_kernel(const unsigned char* __restrict__ dy, const unsigned char* __restrict__ x, int64_t T,
-                     int64_t nvec, const int32_t* __restrict__ cu, int32_t num_seqs, const float* __restrict__ w,
-                     int dilation, int64_t chunk, unsigned char* __restrict__ dx, float* __restrict__ part,
-                     unsigned int* status) {
+__global__ void __launch_bounds__(kConvThreads, dx_min_blocks(K))
+conv_dx_kernel(const unsigned char* __restrict__ dy, int64_t T, int64_t nvec, const int32_t* __restrict__ cu,
+               int32_t num_seqs, const float* __restrict__ w, int dilation, unsigned char* __restrict__ dx,
+               unsigned int* status) {
   constexpr int V = Vec<BF16>::n;
+  constexpr int U = 2 * K;  // chain steps per iteration
   check_cu(cu, num_seqs, T, status);
   const int64_t cv = static_cast<int64_t>(blockIdx.y) * kConvThreads + threadIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * chunk;
-  if (cv >= nvec) return;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kConvChunk;
+  if (cv >= nvec || t0 >= T) return;
   const int64_t C = nvec * V, row = C * (BF16 ? 2 : 4);
-  float wr[V][K], gw[V][K], gb[V];
+  float wr[V][K];
 #pragma unroll
-  for (int v = 0; v < V; ++v) {
-    gb[v] = 0.f;
+  for (int v = 0; v < V; ++v)
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-      wr[v][k] = __ldg(w + (cv * V + v) * K + k);
-      gw[v][k] = 0.f;
-    }
-  }
-  const int64_t t1 = min(T, t0 + chunk), d = dilation;
-  const unsigned char* xc = x + cv * 16;
+    for (int k = 0; k < K; ++k) wr[v][k] = __ldg(w + (cv * V + v) * K + k);
+  const int64_t t1 = min(T, t0 + kConvChunk), d = dilation;
   const unsigned char* gc = dy + cv * 16;
+  unsigned char* dxc = dx + cv * 16;
   Segment sg{cu, num_seqs, 0, T, 0, 0};
-  // each chain's tokens in ascending order, chains in ascending residue: the
-  // order of the partial sums (a fixed function of the sizes)
   for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
     sg.start(t0 + r);
-    uint4 xp[K], xn[K], gn[K], ga[K];  // x: previous / current steps; dy: current / K steps ahead
+    uint4 cur[U], nxt[U];  // dy of this iteration's steps and of the next U steps
 #pragma unroll
-    for (int j = 1; j < K; ++j) {
-      const int64_t t = t0 + r - static_cast<int64_t>(K - j) * d;
-      xp[j] = t >= 0 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int m = 0; m < K; ++m) {
+    for (int m = 0; m < U; ++m) {
       const int64_t t = t0 + r + m * d;
-      gn[m] = t < T ? ld_vec(gc + t * row) : make_uint4(0, 0, 0, 0);
+      cur[m] = t < T ? ld_vec(gc + t * row) : make_uint4(0, 0, 0, 0);
     }
-    for (int64_t tb = t0 + r; tb < t1; tb += K * d) {
+    for (int64_t tb = t0 + r; tb < t1; tb += U * d) {
 #pragma unroll
-      for (int m = 0; m < K; ++m) {
-        const int64_t t = tb + m * d, ta = t + K * d;
-        xn[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
-        ga[m] = ta < T && t < t1 ? ld_vec(gc + ta * row) : make_uint4(0, 0, 0, 0);
+      for (int m = 0; m < U; ++m) {  // K-1 of them are read now, all of them next iteration
+        const int64_t t = tb + (U + m) * d;
+        nxt[m] = t < T && tb + m * d < t1 ? ld_vec(gc + t * row) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int m = 0; m < K; ++m) {
+      for (int m = 0; m < U; ++m) {
         const int64_t t = tb + m * d;
         if (t < t1) {
           sg.advance(t);
-          const int64_t seg_lo = sg.first(t), seg_hi = sg.end(t);
-          float g[V];
-          unpack<BF16>(gn[m], g);
-#pragma unroll
-          for (int v = 0; v < V; ++v) gb[v] += g[v];
+          const int64_t seg_hi = sg.end(t);
           float acc[V];
 #pragma unroll
           for (int v = 0; v < V; ++v) acc[v] = 0.f;
 #pragma unroll
           for (int k = 0; k < K; ++k) {
-            const int j = K - 1 - k;  // chain steps
+            const int j = K - 1 - k;  // chain steps ahead
+            if (t + j * d < seg_hi) {  // x[t] fed output t + j d through tap k
+              float gv[V];
+              unpack<BF16>(m + j < U ? cur[m + j] : nxt[m + j - U], gv);
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+            }
+          }
+          st_cs(dxc + t * row, pack<BF16>(acc));
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < U; ++m) cur[m] = nxt[m];
+    }
+  }
+}
+
+// dweight / dbias of the backward: this chunk's partial sums, written to
+// part[chunk][K + 1][c] (tap k in row k, the bias in row K).  Residue chains again:
+// output t read x at chain steps 0..K-1 back; per 2K chain steps a thread
+// loads the 2K rows of dy and of x, the K-1 x rows before them come from the
+// previous iteration.  The order of a chunk's sum: class by class modulo the
+// dilation, each class in ascending tokens (a fixed function of the sizes).
+template <bool BF16, int K>
+__global__ void __launch_bounds__(kConvThreads, dw_min_blocks(K))
+conv_dw_kernel(const unsigned char* __restrict__ dy, const unsigned char* __restrict__ x, int64_t T, int64_t nvec,
+               const int32_t* __restrict__ cu, int32_t num_seqs, int dilation, int64_t chunk,
+               float* __restrict__ part, unsigned int* status) {
+  constexpr int V = Vec<BF16>::n;
+  constexpr int U = 2 * K;
+  check_cu(cu, num_seqs, T, status);
+  const int64_t cv = static_cast<int64_t>(blockIdx.y) * kConvThreads + threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  if (cv >= nvec) return;
+  const int64_t C = nvec * V, row = C * (BF16 ? 2 : 4);
+  float gw[V][K], gb[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    gb[v] = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) gw[v][k] = 0.f;
+  }
+  const int64_t t1 = min(T, t0 + chunk), d = dilation;
+  const unsigned char* xc = x + cv * 16;
+  const unsigned char* gc = dy + cv * 16;
+  Segment sg{cu, num_seqs, 0, T, 0, 0};
+  for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
+    sg.start(t0 + r);
+    uint4 xp[K], xn[U], gn[U];  // x: the K steps before / this iteration's steps; dy: this iteration's steps
+#pragma unroll
+    for (int j = 1; j < K; ++j) {
+      const int64_t t = t0 + r - static_cast<int64_t>(K - j) * d;
+      xp[j] = t >= 0 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+    }
+    for (int64_t tb = t0 + r; tb < t1; tb += U * d) {
+#pragma unroll
+      for (int m = 0; m < U; ++m) {
+        const int64_t t = tb + m * d;
+        xn[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
+        gn[m] = t < t1 ? ld_vec(gc + t * row) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int m = 0; m < U; ++m) {
+        const int64_t t = tb + m * d;
+        if (t < t1) {
+          sg.advance(t);
+          const int64_t seg_lo = sg.first(t);
+          float g[V];
+          unpack<BF16>(gn[m], g);
+#pragma unroll
+          for (int v = 0; v < V; ++v) gb[v] += g[v];
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const int j = K - 1 - k;  // chain steps back
             if (t - j * d >= seg_lo) {  // output t read x[t - j d] through tap k
               float xv[V];
               unpack<BF16>(m - j >= 0 ? xn[m - j] : xp[K + m - j], xv);
 #pragma unroll
               for (int v = 0; v < V; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
             }
-            if (dx != nullptr && t + j * d < seg_hi) {  // x[t] fed output t + j d through tap k
-              float gv[V];
-              unpack<BF16>(m + j < K ? gn[m + j] : ga[m + j - K], gv);
-#pragma unroll
-              for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
-            }
           }
-          if (dx != nullptr) st_cs(dx + t * row + cv * 16, pack<BF16>(acc));
         }
       }
 #pragma unroll
-      for (int m = 0; m < K; ++m) {
-        xp[m] = xn[m];
-        gn[m] = ga[m];
-      }
+      for (int m = 0; m < K; ++m) xp[m] = xn[U - K + m];
     }
   }
-  if (part == nullptr) return;  // dx only
-  float* pc = part + static_cast<int64_t>(blockIdx.x) * C * (K + 1);
+  float* pc = part + static_cast<int64_t>(blockIdx.x) * C * (K + 1) + cv * V;
 #pragma unroll
-  for (int v = 0; v < V; ++v) {
-    const int64_t c = cv * V + v;
+  for (int k = 0; k <= K; ++k) {  // V consecutive floats per row: coalesced across the warp
 #pragma unroll
-    for (int k = 0; k < K; ++k) pc[c * (K + 1) + k] = gw[v][k];
-    pc[c * (K + 1) + K] = gb[v];
+    for (int v = 0; v < V; v += 4)
+      *reinterpret_cast<float4*>(pc + k * C + v) =
+          k < K ? make_float4(gw[v][k], gw[v + 1][k], gw[v + 2][k], gw[v + 3][k])
+                : make_float4(gb[v], gb[v + 1], gb[v + 2], gb[v + 3]);
   }
 }
 
@@ -289,16 +344,16 @@ __global__ void conv_reduce_kernel(const float* __restrict__ part, int64_t nchun
   wait_for_prior_grid();
   float sum = part[e];
   int64_t q = 1;
-  for (; q + 8 <= nchunks; q += 8) {  // eight loads in flight, added in order
-    float v[8];
+  for (; q < nchunks; q += 32) {  // up to 32 loads in flight, added in order
+    float v[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = part[(q + u) * n + e];
+    for (int u = 0; u < 32; ++u) v[u] = q + u < nchunks ? __ldcs(part + (q + u) * n + e) : 0.f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) sum += v[u];
+    for (int u = 0; u < 32; ++u)
+      if (q + u < nchunks) sum += v[u];
   }
-  for (; q < nchunks; ++q) sum += part[q * n + e];
-  const int64_t c = e / (K + 1);
-  const int k = static_cast<int>(e - c * (K + 1));
+  const int k = static_cast<int>(e / C);  // part[q] is [K + 1][C]
+  const int64_t c = e - k * C;
   if (k < K) {
     if (dw != nullptr) dw[c * K + k] += sum;
   } else if (db != nullptr) {
@@ -404,20 +459,32 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
   const bool bf = dtype == PLE_BF16;
   const int64_t nvec = C / (bf ? 8 : 4);
   const int64_t chunk = conv_chunk_bwd(T), nchunks = conv_chunks_bwd(T);
-  const dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>((nvec + kConvThreads - 1) / kConvThreads));
+  const unsigned vblocks = static_cast<unsigned>((nvec + kConvThreads - 1) / kConvThreads);
   const auto s = static_cast<cudaStream_t>(stream);
-  float* part = want_params ? static_cast<float*>(workspace) : nullptr;  // partial sums only when asked for
+  float* part = static_cast<float*>(workspace);
   const auto* g = static_cast<const unsigned char*>(dy);
   const auto* xb = static_cast<const unsigned char*>(x);
   auto* dxb = static_cast<unsigned char*>(dx);
-#define PLE_CONV_BWD(KK)                                                                                     \
-  case KK:                                                                                                   \
-    if (bf)                                                                                                  \
-      conv_backward_kernel<true, KK><<<grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs, weight, \
-                                                                    dilation, chunk, dxb, part, status);      \
-    else                                                                                                     \
-      conv_backward_kernel<false, KK><<<grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs,      \
-                                                                     weight, dilation, chunk, dxb, part, status); \
+  const dim3 dx_grid(static_cast<unsigned>((T + kConvChunk - 1) / kConvChunk), vblocks);
+  const dim3 dw_grid(static_cast<unsigned>(nchunks), vblocks);
+#define PLE_CONV_BWD(KK)                                                                                          \
+  case KK:                                                                                                        \
+    if (dx != nullptr) {                                                                                          \
+      if (bf)                                                                                                     \
+        conv_dx_kernel<true, KK><<<dx_grid, kConvThreads, 0, s>>>(g, T, nvec, cu_seqlens, num_seqs, weight,       \
+                                                                  dilation, dxb, status);                         \
+      else                                                                                                        \
+        conv_dx_kernel<false, KK><<<dx_grid, kConvThreads, 0, s>>>(g, T, nvec, cu_seqlens, num_seqs, weight,      \
+                                                                   dilation, dxb, status);                        \
+    }                                                                                                             \
+    if (want_params) {                                                                                            \
+      if (bf)                                                                                                     \
+        conv_dw_kernel<true, KK><<<dw_grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs, dilation, \
+                                                                  chunk, part, status);                           \
+      else                                                                                                        \
+        conv_dw_kernel<false, KK><<<dw_grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs,          \
+                                                                   dilation, chunk, part, status);                \
+    }                                                                                                             \
     break;
   switch (K) {
     PLE_CONV_BWD(1) PLE_CONV_BWD(2) PLE_CONV_BWD(3) PLE_CONV_BWD(4)
