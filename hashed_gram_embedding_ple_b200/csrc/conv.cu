@@ -18,6 +18,8 @@
 // (deterministic) and adds the result once into the caller's dw and db.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace ple {
@@ -35,6 +37,9 @@ constexpr int kMaxTaps = 8;
 constexpr int fwd_min_blocks(int K) { return K <= 4 ? 5 : K <= 5 ? 4 : K <= 7 ? 3 : 2; }
 constexpr int dx_min_blocks(int K) { return K <= 4 ? 4 : K <= 7 ? 3 : 2; }
 constexpr int dw_min_blocks(int K) { return K <= 4 ? 4 : K <= 5 ? 3 : 2; }
+constexpr int bwd_min_blocks(int K, bool bf16) {
+  return bf16 ? (K <= 4 ? 4 : K <= 6 ? 3 : 2) : (K <= 2 ? 4 : K <= 4 ? 3 : 2);
+}
 
 template <bool BF16>
 struct Vec {
@@ -72,6 +77,49 @@ __device__ __forceinline__ uint4 pack(const float* v) {
 
 __device__ __forceinline__ uint4 ld_vec(const unsigned char* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
+// Four channels: 8 bytes of bf16 or 16 bytes of fp32 (the fused backward's
+// unit, half the registers per row of a 16-byte bf16 vector).
+template <bool BF16>
+struct Quad {
+  using type = typename std::conditional<BF16, uint2, uint4>::type;
+  static constexpr int bytes = BF16 ? 8 : 16;
+};
+
+template <bool BF16>
+__device__ __forceinline__ typename Quad<BF16>::type ld_quad(const unsigned char* p) {
+  return __ldg(reinterpret_cast<const typename Quad<BF16>::type*>(p));
+}
+
+template <bool BF16>
+__device__ __forceinline__ typename Quad<BF16>::type zero_quad() {
+  typename Quad<BF16>::type z;
+  if constexpr (BF16) z = make_uint2(0, 0); else z = make_uint4(0, 0, 0, 0);
+  return z;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void unpack4(const typename Quad<BF16>::type& u, float* v) {
+  if constexpr (BF16) {
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void st_quad(unsigned char* p, const float* v) {
+  if constexpr (BF16) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    const uint2 u = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+    asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(u.x), "r"(u.y) : "memory");
+  } else {
+    st_cs(p, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3])));
+  }
+}
+
 // The packed segment of the positions a thread walks (in increasing order).
 // Bounds are clamped to [0, T]; with a malformed cu_seqlens (flagged by
 // check_cu) a position the array does not cover is treated as a segment of
@@ -101,6 +149,30 @@ struct Segment {
   }
   __device__ int64_t first(int64_t t) const { return t >= lo && t < hi ? lo : t; }    // history starts here
   __device__ int64_t end(int64_t t) const { return t >= lo && t < hi ? hi : t + 1; }  // lookahead ends here
+};
+
+// The taps of chain position t that stay inside t's segment: `back` chain
+// steps before t (capped at K-1) and `ahead` steps after it (capped).  Kept
+// incrementally along a chain; a division only when the chain enters a
+// segment.  Equivalent to t - j d >= first(t) and t + j d < end(t).
+template <int K>
+struct ChainTaps {
+  int64_t lo = 1, hi = 0, rem = 0;  // segment [lo, hi) of the last step; chain steps left in it
+  int back = 0, ahead = 0;
+  __device__ __forceinline__ void step(Segment& sg, int64_t t, int64_t d) {
+    if (t >= lo && t < hi) {  // one chain step further inside the same segment
+      back = min(back + 1, K - 1);
+      --rem;
+      ahead = rem < K - 1 ? static_cast<int>(rem) : K - 1;
+    } else {
+      sg.advance(t);
+      lo = sg.first(t);
+      hi = sg.end(t);
+      back = static_cast<int>(min((t - lo) / d, static_cast<int64_t>(K - 1)));
+      rem = (hi - 1 - t) / d;
+      ahead = static_cast<int>(min(rem, static_cast<int64_t>(K - 1)));
+    }
+  }
 };
 
 // Block (0, 0) checks cu_seqlens once per launch: cu[0] == 0, cu[S] == T,
@@ -335,6 +407,122 @@ conv_dw_kernel(const unsigned char* __restrict__ dy, const unsigned char* __rest
   }
 }
 
+// The whole backward in one sweep (dx and this chunk's dweight / dbias
+// partials), dy and x each read once.  A thread holds four channels (half a
+// 16-byte bf16 vector, so that the rows of both tensors, both rings and the
+// weight-gradient accumulators fit the register budget of four blocks per
+// SM).  Along a residue chain, K steps per iteration: x at steps -(K-1) ..
+// K-1 and dy at steps 0 .. 2K-2 of the iteration, and the next iteration's
+// rows already in flight.  dx and the partial sums
+// come out bit-identical to conv_dx_kernel and conv_dw_kernel (same
+// per-output tap order, same per-chunk token order).
+template <bool BF16, int K>
+__global__ void __launch_bounds__(kConvThreads, bwd_min_blocks(K, BF16))
+conv_backward_kernel(const unsigned char* __restrict__ dy, const unsigned char* __restrict__ x, int64_t T,
+                     int64_t nquad, const int32_t* __restrict__ cu, int32_t num_seqs, const float* __restrict__ w,
+                     int dilation, int64_t chunk, unsigned char* __restrict__ dx, float* __restrict__ part,
+                     unsigned int* status) {
+  using Q = typename Quad<BF16>::type;
+  constexpr int U = K, L = K - 1, LS = L > 0 ? L : 1;
+  check_cu(cu, num_seqs, T, status);
+  const int64_t cq = static_cast<int64_t>(blockIdx.y) * kConvThreads + threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  if (cq >= nquad) return;
+  const int64_t C = nquad * 4, row = C * (BF16 ? 2 : 4);
+  float wr[4][K], gw[4][K], gb[4];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    gb[v] = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      wr[v][k] = __ldg(w + (cq * 4 + v) * K + k);
+      gw[v][k] = 0.f;
+    }
+  }
+  const int64_t t1 = min(T, t0 + chunk), d = dilation;
+  const unsigned char* xc = x + cq * Quad<BF16>::bytes;
+  const unsigned char* gc = dy + cq * Quad<BF16>::bytes;
+  unsigned char* dxc = dx + cq * Quad<BF16>::bytes;
+  Segment sg{cu, num_seqs, 0, T, 0, 0};
+  for (int64_t r = 0; r < d && t0 + r < t1; ++r) {
+    sg.start(t0 + r);
+    ChainTaps<K> ct;
+    // x at steps -L .. -1 (xp) and 0 .. U-1 (xn); dy at steps 0 .. L-1 (ga) and L .. L+U-1 (gn)
+    Q xp[LS], ga[LS], xn[U], gn[U];
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+      const int64_t tx = t0 + r - static_cast<int64_t>(L - i) * d, tg = t0 + r + i * d;
+      xp[i] = tx >= 0 ? ld_quad<BF16>(xc + tx * row) : zero_quad<BF16>();
+      ga[i] = tg < T ? ld_quad<BF16>(gc + tg * row) : zero_quad<BF16>();
+    }
+#pragma unroll
+    for (int m = 0; m < U; ++m) {
+      const int64_t t = t0 + r + m * d, tg = t0 + r + (L + m) * d;
+      xn[m] = t < t1 ? ld_quad<BF16>(xc + t * row) : zero_quad<BF16>();
+      gn[m] = tg < T && t < t1 ? ld_quad<BF16>(gc + tg * row) : zero_quad<BF16>();
+    }
+    for (int64_t tb = t0 + r; tb < t1; tb += U * d) {
+      Q xq[U], gq[U];  // the next iteration's rows, in flight during this one's arithmetic
+#pragma unroll
+      for (int m = 0; m < U; ++m) {
+        const int64_t t = tb + (U + m) * d, tg = tb + (U + L + m) * d;
+        xq[m] = t < t1 ? ld_quad<BF16>(xc + t * row) : zero_quad<BF16>();
+        gq[m] = tg < T && t < t1 ? ld_quad<BF16>(gc + tg * row) : zero_quad<BF16>();
+      }
+#pragma unroll
+      for (int m = 0; m < U; ++m) {
+        const int64_t t = tb + m * d;
+        if (t < t1) {
+          ct.step(sg, t, d);
+          float g[4];
+          unpack4<BF16>(m < L ? ga[m] : gn[m - L], g);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) gb[v] += g[v];
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const int j = K - 1 - k;
+            if (j <= ct.back) {  // output t read x[t - j d] through tap k
+              float xv[4];
+              unpack4<BF16>(m - j >= 0 ? xn[m - j] : xp[L + m - j], xv);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
+            }
+          }
+          if (dx != nullptr) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+              const int j = K - 1 - k;
+              if (j <= ct.ahead) {  // x[t] fed output t + j d through tap k
+                float gv[4];
+                unpack4<BF16>(m + j < L ? ga[m + j] : gn[m + j - L], gv);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+              }
+            }
+            st_quad<BF16>(dxc + t * row, acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < L; ++i) {
+        xp[i] = xn[U - L + i];
+        ga[i] = gn[U - L + i];
+      }
+#pragma unroll
+      for (int m = 0; m < U; ++m) {
+        xn[m] = xq[m];
+        gn[m] = gq[m];
+      }
+    }
+  }
+  float* pc = part + static_cast<int64_t>(blockIdx.x) * C * (K + 1) + cq * 4;
+#pragma unroll
+  for (int k = 0; k <= K; ++k)
+    *reinterpret_cast<float4*>(pc + k * C) =
+        k < K ? make_float4(gw[0][k], gw[1][k], gw[2][k], gw[3][k]) : make_float4(gb[0], gb[1], gb[2], gb[3]);
+}
+
 // dw[c, k] += sum over chunks (in chunk order) of the partials; db likewise.
 __global__ void conv_reduce_kernel(const float* __restrict__ part, int64_t nchunks, int64_t C, int K,
                                    float* __restrict__ dw, float* __restrict__ db) {
@@ -467,17 +655,28 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
   auto* dxb = static_cast<unsigned char*>(dx);
   const dim3 dx_grid(static_cast<unsigned>((T + kConvChunk - 1) / kConvChunk), vblocks);
   const dim3 dw_grid(static_cast<unsigned>(nchunks), vblocks);
+  const int64_t nquad = C / 4;
+  const dim3 fused_grid(static_cast<unsigned>(nchunks),
+                        static_cast<unsigned>((nquad + kConvThreads - 1) / kConvThreads));
 #define PLE_CONV_BWD(KK)                                                                                          \
   case KK:                                                                                                        \
-    if (dx != nullptr) {                                                                                          \
+    if (dx != nullptr && want_params) {                                                                           \
+      if (bf)                                                                                                     \
+        conv_backward_kernel<true, KK><<<fused_grid, kConvThreads, 0, s>>>(g, xb, T, nquad, cu_seqlens, num_seqs, \
+                                                                           weight, dilation, chunk, dxb, part,    \
+                                                                           status);                               \
+      else                                                                                                        \
+        conv_backward_kernel<false, KK><<<fused_grid, kConvThreads, 0, s>>>(g, xb, T, nquad, cu_seqlens,          \
+                                                                            num_seqs, weight, dilation, chunk,    \
+                                                                            dxb, part, status);                   \
+    } else if (dx != nullptr) {                                                                                   \
       if (bf)                                                                                                     \
         conv_dx_kernel<true, KK><<<dx_grid, kConvThreads, 0, s>>>(g, T, nvec, cu_seqlens, num_seqs, weight,       \
                                                                   dilation, dxb, status);                         \
       else                                                                                                        \
         conv_dx_kernel<false, KK><<<dx_grid, kConvThreads, 0, s>>>(g, T, nvec, cu_seqlens, num_seqs, weight,      \
                                                                    dilation, dxb, status);                        \
-    }                                                                                                             \
-    if (want_params) {                                                                                            \
+    } else {                                                                                                      \
       if (bf)                                                                                                     \
         conv_dw_kernel<true, KK><<<dw_grid, kConvThreads, 0, s>>>(g, xb, T, nvec, cu_seqlens, num_seqs, dilation, \
                                                                   chunk, part, status);                           \

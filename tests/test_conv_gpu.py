@@ -73,6 +73,15 @@ def run_case(dev, lens, C, K, d, dt, seed=0, with_bias=True):
     assert torch.equal(dbt2.view(torch.int32), dbt.view(torch.int32))
     assert torch.equal(dx2.view(torch.int16 if dt == synth.DTYPE_BF16 else torch.int32),
                        dx.view(torch.int16 if dt == synth.DTYPE_BF16 else torch.int32))
+    # dx with the parameter gradients runs as one sweep, each alone as its own
+    # kernel: the same sums in the same order, bit for bit
+    dx3, _, _ = ple.conv_backward(gt, xt, cut, wt, d)
+    dwt3, dbt3 = torch.from_numpy(dw0.copy()).to(dev), torch.from_numpy(db0.copy()).to(dev)
+    ple.conv_backward(gt, xt, cut, wt, d, want_dx=False, dweight=dwt3, dbias=dbt3)
+    assert torch.equal(dx3.view(torch.int16 if dt == synth.DTYPE_BF16 else torch.int32),
+                       dx.view(torch.int16 if dt == synth.DTYPE_BF16 else torch.int32))
+    assert torch.equal(dwt3.view(torch.int32), dwt.view(torch.int32))
+    assert torch.equal(dbt3.view(torch.int32), dbt.view(torch.int32))
 
 
 @pytest.mark.parametrize("C,K,d,dt", [
