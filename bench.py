@@ -581,9 +581,7 @@ def run_conv(args, rank, world, dev, dist):
     e = 2
     nchunks = max(1, -(-ws.numel() // (C * (K + 1) * 4)))
     fwd_bytes = 2 * T * C * e                                     # x read, y written
-    # dy and x read, dx written; partial sums (the least a backward moves: the
-    # dx and dweight kernels each read dy, which traffic shows and this does not count)
-    bwd_bytes = 3 * T * C * e + 2 * nchunks * C * (K + 1) * 4
+    bwd_bytes = 3 * T * C * e + 2 * nchunks * C * (K + 1) * 4    # dy and x read, dx written; partial sums
     fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
     bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9
     src = ["hashed_gram_embedding_ple_b200/csrc/conv.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
@@ -594,7 +592,7 @@ def run_conv(args, rank, world, dev, dist):
     roof_b = {"bound": "hbm", "achieved": bwd_gbs, "peak": peak, "unit": "GB/s", "frac": bwd_gbs / peak,
               "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": bwd_bytes,
               "traffic": traffic_from_profiles("conv_backward_conv_single_layer", src),
-              "kernel": "conv_dx_kernel + conv_dw_kernel + conv_reduce_kernel", "peak_source": f"{peak_kind} hbm_gbs"}
+              "kernel": "conv_backward_kernel + conv_reduce_kernel", "peak_source": f"{peak_kind} hbm_gbs"}
     roofline = roof_b if ms_bwd > ms_fwd else roof_f
 
     e2e = None
@@ -659,7 +657,7 @@ def run_conv(args, rank, world, dev, dist):
                 "bwd": {"ms": ms_bwd, "gb_per_s": bwd_gbs, "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS,
                         "frac_of_measured": bwd_gbs / peak},
                 "roofline": roofline, "roofline_fwd": roof_f, "roofline_bwd": roof_b, "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clocks, "wall_s_timed_region": wall}
+                "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks, "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
