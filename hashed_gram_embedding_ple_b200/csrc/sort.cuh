@@ -47,7 +47,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // ---------------------------------------------------------------------------
 constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
-constexpr int kSortItems = 8;
+constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortThreads * kSortItems;  // positions per tile
 constexpr int kWarpSpan = kSortTile / kSortWarps;     // positions per warp within a tile
 constexpr int kMaxPasses = 4;
@@ -234,7 +234,7 @@ key_hist_kernel(const int64_t* __restrict__ rows, int64_t num_rows, const SortAr
   allow_next_grid();
 }
 
-__global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortArgs a, const int pass) {
+__global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortArgs a, const int pass) {
   __shared__ uint32_t wh[kSortWarps][kRadix];
   __shared__ uint32_t stage_k[kSortTile];
   __shared__ uint32_t stage_v[kSortTile];
@@ -297,14 +297,14 @@ __global__ void __launch_bounds__(kSortThreads, 3) sort_pass_kernel(const SortAr
   for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
   __syncthreads();
   // rank among the same digit within the warp's positions, in order
-  uint8_t rank[kSortItems];
+  uint16_t rank[kSortItems];
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
     const bool valid = i0 + r * 32 + lane < N;
     const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
     const unsigned peers = peers_of<8>(valid, digit);
     const unsigned lower = __popc(peers & lanemask_lt());
-    rank[r] = valid ? static_cast<uint8_t>(wh[warp][digit] + lower) : 0;  // < 256 keys per warp
+    rank[r] = valid ? static_cast<uint16_t>(wh[warp][digit] + lower) : 0;  // < 512 keys per warp
     __syncwarp();
     if (valid && lower == 0) wh[warp][digit] += __popc(peers);
     __syncwarp();
