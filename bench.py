@@ -439,17 +439,33 @@ def main():
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         d_tok, d_cu = torch.empty_like(tokens), torch.empty_like(cu)
         d_grad = torch.empty_like(grad) if do_bwd else None
+        # the link is full duplex: grad_out goes up on one copy stream from the
+        # step's start, the lookup output comes down on another as soon as the
+        # lookup is done, while the backward runs on the compute stream
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_start, ev_fwd, ev_up, ev_down = (torch.cuda.Event() for _ in range(4))
         times = []
         for k in range(args.e2e_steps + 2):
             flush_l2()
             e0.record(stream)
+            ev_start.record(stream)
+            if do_bwd:
+                up.wait_event(ev_start)
+                with torch.cuda.stream(up):
+                    d_grad.copy_(h_grad, non_blocking=True)
+                    ev_up.record(up)
             d_tok.copy_(h_tok, non_blocking=True)
             d_cu.copy_(h_cu, non_blocking=True)
             lookup(d_tok, d_cu)
+            ev_fwd.record(stream)
+            down.wait_event(ev_fwd)
+            with torch.cuda.stream(down):
+                h_out.copy_(out, non_blocking=True)
+                ev_down.record(down)
             if do_bwd:
-                d_grad.copy_(h_grad, non_blocking=True)
+                stream.wait_event(ev_up)
                 ple.ple_grad_scatter(plan, rows.view(-1), d_grad, table_grad, workspace=ws)
-            h_out.copy_(out, non_blocking=True)
+            stream.wait_event(ev_down)
             e1.record(stream)
             torch.cuda.synchronize()
             if k >= 2:
@@ -458,7 +474,9 @@ def main():
         h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
         e2e = {"value": world * T / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": N_out * D * e_o, "ms_per_step": t_e2e_ms,
-               "what": "pinned H2D tokens+cu_seqlens+grad_out, ple_lookup, ple_grad_scatter, D2H of the lookup output"}
+               "what": "pinned H2D tokens+cu_seqlens, ple_lookup, D2H of the lookup output; H2D of grad_out on a "
+                       "second copy stream from the step's start, then ple_grad_scatter; the D2H on a third stream "
+                       "beside it (full-duplex link); all inside the CUDA events"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and sl is None:
@@ -601,16 +619,33 @@ def run_conv(args, rank, world, dev, dist):
         hy, hdx = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
         dxin, dgin = torch.empty_like(x), torch.empty_like(g)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # x goes up first; dy follows on a copy stream while the forward runs,
+        # y comes down on another while dy goes up (full-duplex link), then dx
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_x, ev_y, ev_g, ev_dx, ev_down = (torch.cuda.Event() for _ in range(5))
         times = []
         for k in range(args.e2e_steps + 1):
             flush_l2()
             e0.record(stream)
             dxin.copy_(hx, non_blocking=True)
-            dgin.copy_(hg, non_blocking=True)
+            ev_x.record(stream)
+            up.wait_event(ev_x)
+            with torch.cuda.stream(up):
+                dgin.copy_(hg, non_blocking=True)
+                ev_g.record(up)
             fwd(dxin)
+            ev_y.record(stream)
+            down.wait_event(ev_y)
+            with torch.cuda.stream(down):
+                hy.copy_(y, non_blocking=True)
+            stream.wait_event(ev_g)
             bwd(dgin, dxin)
-            hy.copy_(y, non_blocking=True)
-            hdx.copy_(dx, non_blocking=True)
+            ev_dx.record(stream)
+            down.wait_event(ev_dx)
+            with torch.cuda.stream(down):
+                hdx.copy_(dx, non_blocking=True)
+                ev_down.record(down)
+            stream.wait_event(ev_down)
             e1.record(stream)
             torch.cuda.synchronize()
             if k >= 1:
@@ -618,7 +653,9 @@ def run_conv(args, rank, world, dev, dist):
         (t_e2e,) = reduce_max([statistics.mean(times)], dist, dev)
         e2e = {"value": world * T / (t_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 2 * T * C * e,
                "d2h_bytes_per_step": 2 * T * C * e, "ms_per_step": t_e2e,
-               "what": "pinned H2D of x and dy, ple_conv_forward, ple_conv_backward, D2H of y and dx"}
+               "what": "pinned H2D of x, ple_conv_forward, D2H of y; H2D of dy on a copy stream after x, "
+                       "ple_conv_backward, D2H of dx; D2H on a third stream (full-duplex link); all inside the "
+                       "CUDA events"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
