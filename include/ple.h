@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   PLE_OK = 0,
   PLE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad constants */
-  PLE_ERR_UNSUPPORTED = 2,   /* a limit of this build (see each entry) */
+  PLE_ERR_UNSUPPORTED = 2,   /* a limit of this library (see each entry) */
   PLE_ERR_ALIGNMENT = 3,     /* pointer or row size not 16-byte aligned */
   PLE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
   PLE_ERR_CUDA = 5,          /* CUDA runtime error; see ple_last_cuda_error */
