@@ -278,19 +278,15 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
   __syncthreads();
   const uint32_t count = tid < kRadix ? start_s[tid] : 0;  // keys of digit tid in this tile
   if (tid < kRadix) st_relaxed(tile_rows + t * kRadix + tid, kReady | count);
-  // keys of digit tid in the earlier tiles, over the three levels (wh is the scratch)
-  {
-    uint32_t* group_rows = tile_rows + a.tiles * kRadix;
-    uint32_t* super_rows = group_rows + a.groups * kRadix;
-    const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
-    uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
-    if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
-    before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
-    if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
-    before += level_sum(super_rows, 0, sg, wh, a.status);
-    if (tid < kRadix) base_s[tid] += before;
-  }
-  // tile-local start of every digit
+  // keys of digit tid in the earlier tiles of its group (wh is the scratch),
+  // so that the group's total is published early
+  uint32_t* group_rows = tile_rows + a.tiles * kRadix;
+  uint32_t* super_rows = group_rows + a.groups * kRadix;
+  const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
+  uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
+  if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
+  // then everything local to the tile (its ranks, the tile staged in digit
+  // order) while the other groups' totals are published
   uint32_t tile_n;
   const uint32_t local_start = block_exclusive_sum(count, warp_tot, &tile_n);
   if (tid < kRadix) start_s[tid] = local_start;
@@ -320,8 +316,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
     }
   }
   __syncthreads();
-  // stage the tile in digit order, then coalesced writes: consecutive
-  // threads, consecutive destinations within a digit
+  // stage the tile in digit order (consecutive positions within a digit)
 #pragma unroll
   for (int r = 0; r < kSortItems; ++r) {
     if (i0 + r * 32 + lane < N) {
@@ -332,6 +327,13 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
     }
   }
   __syncthreads();
+  // keys of digit tid in the earlier groups and supergroups (wh is the scratch again)
+  before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
+  if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
+  before += level_sum(super_rows, 0, sg, wh, a.status);
+  if (tid < kRadix) base_s[tid] += before;
+  __syncthreads();
+  // coalesced writes: consecutive threads, consecutive destinations within a digit
   for (uint32_t j = tid; j < tile_n; j += kSortThreads) {
     const uint32_t k2 = stage_k[j];
     const uint32_t digit = (k2 >> shift) & (kRadix - 1);
