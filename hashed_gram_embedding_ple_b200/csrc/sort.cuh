@@ -27,7 +27,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // key_hist_kernel turns the int64 rows into 32-bit keys and counts the
 // digits of every pass at once, so the global start of each digit is known
 // before the first pass.  Each pass is one sort_pass_kernel launch in which
-// a block takes one tile of kSortTile consecutive positions, in the order of
+// a block takes one tile of consecutive positions, in the order of
 // a ticket counter (a block only ever waits for tiles with lower tickets,
 // whose blocks are already running).  The block ranks its keys by digit
 // (warp ballots, per-warp running counts: stable) and publishes its
@@ -47,9 +47,13 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // ---------------------------------------------------------------------------
 constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
-constexpr int kSortItems = 16;
-constexpr int kSortTile = kSortThreads * kSortItems;  // positions per tile
-constexpr int kWarpSpan = kSortTile / kSortWarps;     // positions per warp within a tile
+// Keys per thread: 16 (4096-key tiles, 2 blocks per SM) from kBigTileKeys
+// keys on, else 8 (2048-key tiles, 3 blocks per SM): fewer tiles shorten the
+// look-back, but below about 3 * 2^17 keys there are too few of them to
+// fill the SMs (measured on the B200: 2048-key tiles win at 262144 keys,
+// 4096-key tiles at 524288 and above).
+constexpr int64_t kBigTileKeys = 3 << 17;
+inline int sort_items(int64_t N) { return N >= kBigTileKeys ? 16 : 8; }
 constexpr int kMaxPasses = 4;
 constexpr int kGroupBits = 5;                         // 32 tiles per group, 32 groups per supergroup
 constexpr unsigned kSpinLimit = 1u << 22;             // a few seconds of polling, then give up
@@ -234,7 +238,10 @@ key_hist_kernel(const int64_t* __restrict__ rows, int64_t num_rows, const SortAr
   allow_next_grid();
 }
 
-__global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortArgs a, const int pass) {
+template <int ITEMS>
+__global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_kernel(const SortArgs a, const int pass) {
+  constexpr int kSortTile = kSortThreads * ITEMS;   // positions per tile
+  constexpr int kWarpSpan = kSortTile / kSortWarps;  // positions per warp within a tile
   __shared__ uint32_t wh[kSortWarps][kRadix];
   __shared__ uint32_t stage_k[kSortTile];
   __shared__ uint32_t stage_v[kSortTile];
@@ -263,9 +270,9 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
   uint32_t* vout = odd ? a.vals[0] : a.vals[1];
   uint32_t* tile_rows = a.look + static_cast<int64_t>(pass) * (a.tiles + a.groups + a.supers) * kRadix;
 
-  uint32_t key[kSortItems], val[kSortItems];
+  uint32_t key[ITEMS], val[ITEMS];
 #pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
+  for (int r = 0; r < ITEMS; ++r) {
     const int64_t i = i0 + r * 32 + lane;
     key[r] = i < N ? kin[i] : 0;
     val[r] = i < N ? (pass == 0 ? static_cast<uint32_t>(i) : vin[i]) : 0;
@@ -273,7 +280,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
   // digit counts of the tile (shared-memory atomics), published at once so
   // that later tiles' look-backs do not wait for this tile's ranking
 #pragma unroll
-  for (int r = 0; r < kSortItems; ++r)
+  for (int r = 0; r < ITEMS; ++r)
     if (i0 + r * 32 + lane < N) atomicAdd(&start_s[(key[r] >> shift) & (kRadix - 1)], 1u);
   __syncthreads();
   const uint32_t count = tid < kRadix ? start_s[tid] : 0;  // keys of digit tid in this tile
@@ -293,9 +300,9 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
   for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
   __syncthreads();
   // rank among the same digit within the warp's positions, in order
-  uint16_t rank[kSortItems];
+  uint16_t rank[ITEMS];
 #pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
+  for (int r = 0; r < ITEMS; ++r) {
     const bool valid = i0 + r * 32 + lane < N;
     const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
     const unsigned peers = peers_of<8>(valid, digit);
@@ -318,7 +325,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) sort_pass_kernel(const SortAr
   __syncthreads();
   // stage the tile in digit order (consecutive positions within a digit)
 #pragma unroll
-  for (int r = 0; r < kSortItems; ++r) {
+  for (int r = 0; r < ITEMS; ++r) {
     if (i0 + r * 32 + lane < N) {
       const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
       const uint32_t pos = start_s[digit] + wh[warp][digit] + rank[r];
@@ -353,12 +360,15 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
 struct SortLayout {
   size_t keys[2], vals[2], look, zeroed, zeroed_bytes;
   int64_t tiles, groups, supers;
+  int items;  // keys per thread of the sort passes
 };
 
 // Places the sort's buffers for N keys at byte offset *off (advanced past them).
 inline SortLayout sort_layout(int64_t N, size_t* off) {
   SortLayout L{};
-  L.tiles = (N + kSortTile - 1) / kSortTile;
+  L.items = sort_items(N);
+  const int64_t tile = static_cast<int64_t>(kSortThreads) * L.items;
+  L.tiles = (N + tile - 1) / tile;
   L.groups = (L.tiles + 31) >> kGroupBits;
   L.supers = (L.groups + 31) >> kGroupBits;
   auto take = [&](size_t bytes) {
@@ -421,7 +431,10 @@ inline ple_status_t launch_sort(const int64_t* rows, int64_t N, int64_t num_rows
                    num_rows, sa, run_done, nwin);
   if (e != cudaSuccess) return cuda_fail(e);
   for (int p = 0; p < sa.passes; ++p) {
-    e = launch_after(sort_pass_kernel, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s, sa, p);
+    e = L.items > 8 ? launch_after(sort_pass_kernel<16>, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s,
+                                   sa, p)
+                    : launch_after(sort_pass_kernel<8>, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s,
+                                   sa, p);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   *sorted_keys = sa.keys[sa.passes & 1];
