@@ -177,6 +177,18 @@ def test_gradient_many_tiles(cuda_device, D, gdt):
     check_backward(w, cuda_device, rows)
 
 
+@pytest.mark.parametrize("N", [3 * 2**17 - 1, 3 * 2**17 + 777])
+def test_gradient_both_sort_tile_sizes(cuda_device, N):
+    """Just below and above the key count at which the sort passes switch
+    from 2048-key to 4096-key tiles (ragged last tile on both sides)."""
+    rng = np.random.default_rng(N)
+    R = 1_000_003
+    rows = synth.zipf_ids(N, 1.2, R, rng)
+    w = custom_workload("gswitch", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [R], 16, synth.DTYPE_F32,
+                        synth.DTYPE_BF16)
+    check_backward(w, cuda_device, rows)
+
+
 def test_bad_rows_flagged(cuda_device):
     dev = cuda_device
     w = synth.tiny(0)
