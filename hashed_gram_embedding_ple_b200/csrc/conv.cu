@@ -12,10 +12,11 @@
 // load and store of a warp covers 512 consecutive bytes of a token row and
 // each row is loaded once (plus K-1 rows of history per class and chunk).
 // The backward pass computes dx (the same taps looking ahead, inside the
-// segment) in one kernel and per-chunk partial sums of dw and db in another
-// (dy is read by both; apart, each keeps few enough registers to have its
-// rows in flight); a third kernel adds the chunk partials in chunk order
-// (deterministic) and adds the result once into the caller's dw and db.
+// segment) and per-chunk partial sums of dw and db in one sweep when both
+// are asked for (dy and x read once; a thread owns 4 channels there so that
+// both tensors' rows fit its registers), or either alone in a kernel of its
+// own; a last kernel adds the chunk partials in chunk order (deterministic)
+// and adds the result once into the caller's dw and db.
 #include <cuda_bf16.h>
 
 #include <type_traits>
