@@ -10,6 +10,7 @@
 //   added once into table_grad[r].
 //
 // Pipeline (all in the caller's workspace, no allocation):
+//   0. clear_kernel: zeroes the digit totals and the tile tickets;
 //   1. key_hist_kernel: 32-bit keys from the int64 rows (bad rows -> key R)
 //      and the digit counts of every radix pass;
 //   2. sort_pass_kernel, once per 8-bit digit: LSD radix sort, stable,

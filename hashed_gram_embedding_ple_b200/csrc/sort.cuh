@@ -27,21 +27,24 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // key_hist_kernel turns the int64 rows into 32-bit keys and counts the
 // digits of every pass at once, so the global start of each digit is known
 // before the first pass.  Each pass is one sort_pass_kernel launch in which
-// a block takes one tile of consecutive positions, in the order of
-// a ticket counter (a block only ever waits for tiles with lower tickets,
-// whose blocks are already running).  The block ranks its keys by digit
-// (warp ballots, per-warp running counts: stable) and publishes its
-// per-digit counts.  The keys of a digit in all earlier tiles are then
-// summed over three levels, so that no tile waits on a long chain:
+// a block takes one tile of consecutive positions (2048 or 4096 keys, by
+// the key count), in the order of a ticket counter (a block only ever waits
+// for tiles with lower tickets, whose blocks are already running).  The
+// block counts its keys per digit and publishes the counts at once.  The
+// keys of a digit in all earlier tiles are summed over three levels, so
+// that no tile waits on a long chain:
 //   tiles of its group of 32 tiles before it (their counts);
 //   groups of its supergroup of 32 groups before its group (group totals,
-//   published by the last tile of each group);
+//   published by the last tile of each group as soon as it has its level);
 //   supergroups before its supergroup (totals published by the last tile of
 //   each supergroup).
+// Between the first level and the other two the block ranks its keys by
+// digit (warp ballots, per-warp running counts: stable) and stages the tile
+// in shared memory in digit order, while the other groups publish.
 // A published word is READY | count; the count is the payload, so plain
 // relaxed loads and stores suffice.  Keys then go to digit start + earlier
-// count + rank, staged in shared memory in digit order so that the writes
-// are coalesced.  Every wait is bounded: past the limit the block raises
+// count + rank, written from the staged tile so that the writes are
+// coalesced.  Every wait is bounded: past the limit the block raises
 // PLE_ERR_TIMEOUT and carries on with what it has (the result is then
 // unspecified; nothing hangs).
 // ---------------------------------------------------------------------------
