@@ -288,8 +288,12 @@ size_t ple_conv_backward_workspace_bytes(int64_t num_tokens, int64_t channels, i
  * The sums over tokens have a fixed order, so results are bit-identical run
  * to run: the tokens are cut into consecutive chunks (at least 256 tokens,
  * at most 1024 chunks); each chunk's sum starts from +0 and adds its tokens
- * in order (fused multiply-add for dweight); the chunk sums are added in
- * chunk order starting from the first; one final add into dweight / dbias.
+ * residue class by residue class modulo the dilation (the class of the
+ * chunk's first token first), each class in ascending token order (fused
+ * multiply-add for dweight); the chunk sums are added in chunk order
+ * starting from the first; one final add into dweight / dbias.  dx and the
+ * parameter gradients come out with the same bits whether they are asked
+ * for together (one sweep) or separately.
  * workspace (16-byte aligned, ple_conv_backward_workspace_bytes) is needed
  * only for dweight or dbias.  Errors as ple_conv_forward, plus
  * PLE_ERR_WORKSPACE. */
