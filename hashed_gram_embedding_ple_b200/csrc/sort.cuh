@@ -381,7 +381,12 @@ inline SortLayout sort_layout(int64_t N, size_t* off) {
   };
   for (int b = 0; b < 2; ++b) L.keys[b] = take(sizeof(uint32_t) * N);
   for (int b = 0; b < 2; ++b) L.vals[b] = take(sizeof(uint32_t) * N);
-  L.look = take(sizeof(uint32_t) * kRadix * kMaxPasses * static_cast<size_t>(L.tiles + L.groups + L.supers));
+  // the look-back rows are sized for the smaller tiles whatever the tiling,
+  // so the workspace never shrinks as N grows (a workspace sized for some N
+  // serves every smaller N)
+  const int64_t small_tiles = (N + kSortThreads * 8 - 1) / (kSortThreads * 8);
+  const int64_t small_groups = (small_tiles + 31) >> kGroupBits, small_supers = (small_groups + 31) >> kGroupBits;
+  L.look = take(sizeof(uint32_t) * kRadix * kMaxPasses * static_cast<size_t>(small_tiles + small_groups + small_supers));
   L.zeroed_bytes = sizeof(uint32_t) * (kMaxPasses * kRadix + kMaxPasses);
   L.zeroed = take(L.zeroed_bytes);
   return L;

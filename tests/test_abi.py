@@ -126,6 +126,19 @@ def test_workspace_grows_with_hits():
     assert b >= 100000 * (16 + 2 * 128 * 4 // 32)
 
 
+def test_workspace_never_shrinks_as_hits_grow():
+    """A workspace sized for N hits serves every smaller N, across the sort's
+    switch from 2048-key to 4096-key tiles (at 3 * 2^17 keys) too."""
+    for D in (16, 64, 128):
+        p = _plan(head_dim=D)
+        ns = sorted({1, 31, 32, 33, 2047, 2048, 2049, 65535, 65536, 3 * 2**17 - 4097, 3 * 2**17 - 1, 3 * 2**17,
+                     3 * 2**17 + 1, 3 * 2**17 + 4096, 524288, 1 << 21, (1 << 21) + 1})
+        sizes = [ple.workspace_bytes(p, n) for n in ns]
+        assert all(a <= b for a, b in zip(sizes, sizes[1:])), list(zip(ns, sizes))
+        host = [ple.lib().ple_prefetch_workspace_bytes(p.handle, n) for n in ns]
+        assert all(a <= b for a, b in zip(host, host[1:]))
+
+
 def test_strerror_covers_codes():
     lib = ple.lib()
     for c in range(9):
