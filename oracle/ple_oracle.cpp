@@ -29,7 +29,11 @@
 //    hits of row r in ascending flat index i = t*H + j, cut into chunks of 32
 //    consecutive hits; each chunk summed left to right starting from its
 //    first element; the chunk sums summed left to right starting from the
-//    first; the result added once into table_grad[r].
+//    first; the result added once into table_grad[r].  Parity unpinned by
+//    the page for that order itself: it is the library's contract, held here
+//    by closed-form cases only this order produces (the pins in
+//    tests/test_oracle_pins.py), while the sums' values are pinned against
+//    fp64 index_add and exact integer gradients.
 //
 // Build: g++ -O2 -ffp-contract=off -std=c++17 -shared -fPIC (no fast-math,
 // so every float add below is one IEEE round-to-nearest add).
