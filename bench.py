@@ -1,14 +1,20 @@
 #!/usr/bin/env python3
 """Throughput of the hashed n-gram (PLE / Engram) lookup on B200.
 
-One step = the whole hot path over one batch of synthetic packed tokens:
+One step = the whole hot path over synthetic packed tokens: for each part
   forward  ple_lookup   (segment/EOS context, order hashes, head rows, row
                          gather; the rows are saved for the backward)
   backward ple_grad_scatter (deterministic table gradient of the gather)
-Default workload: 8 packed sequences totalling 32768 tokens (lengths 1k-8k),
-Zipf(1.1) ids over a 151936-id vocabulary, EOS 0.5 %, ngram_size 3, 8 heads
-per order (16 heads), 16 consecutive primes >= 1e6 (16.0M rows), head_dim 64
-bf16 table (2.05 GB); bf16 grad_out N(0,1) into an fp32 table gradient.
+Default step (--workload headline), the two largest single-GPU workloads:
+  large_table      forward: 65536 tokens (14 packed sequences, 1k-8k),
+                   Zipf(1.1) ids over 151936, EOS 0.5 %, ngram_size 4, 8
+                   heads per order (24 heads), 24 primes >= 8.4e6 (201.6 M
+                   rows), head_dim 128 bf16 table (51.6 GB);
+  backward_stress  forward + backward: 131072 tokens, Zipf(1.3) with
+                   repeated 64-token spans, 16 heads, 16 primes >= 1e6,
+                   head_dim 128, bf16 grad_out N(0,1) into an 8.2 GB fp32
+                   table gradient.
+--workload NAME runs one workload (forward + backward, or --fwd-only).
 
 Prints ONE JSON line on rank 0 (everything else goes to stderr).
 Multi-GPU: the lookup has no exchange step on one node (one GPU holds the
@@ -179,69 +185,181 @@ def replica_seed(base: int, rank: int) -> int:
     return base + rank
 
 
-def cpu_oracle_step(w, table_host, grad_host, threads, tokens_limit=None):
-    """The oracle, as it stands, on the first `tokens_limit` tokens (whole
-    sequences cut at that point): rows, gather, gradient sums."""
+# The default step: the forward on the large-table workload (65536 tokens,
+# 24 heads, D=128, 51.6 GB bf16 table) and the forward + backward on the
+# backward-stress workload (131072 tokens, 16 heads, D=128, Zipf(1.3) with
+# repeated spans, bf16 grad_out into an 8.2 GB fp32 table gradient): the two
+# largest single-GPU configurations, one for each direction.
+HEADLINE = (("large_table", False), ("backward_stress", True))
+
+
+def step_parts(args):
+    """(workload name, with backward) for every part of one step."""
+    if args.workload == "headline":
+        return list(HEADLINE)
+    return [(args.workload, not args.fwd_only)]
+
+
+def compact_table(w, rows, table_rows):
+    """A host table holding only the rows a pass touches, and the rows
+    renumbered into it (the oracle's gather is a copy per hit, so a compact
+    table gives it the same work without a table-sized host array)."""
+    uniq, inv = np.unique(rows, return_inverse=True)
+    return table_rows(uniq), inv.reshape(rows.shape).astype(np.int64)
+
+
+def cpu_oracle_pass(w, tok, cu, table_c, rows_c, grad_host, threads):
+    """The oracle, as it stands: rows, gather (from the compact table) and,
+    with grad_host, the gradient sums.  Returns the seconds taken."""
     import oracle
 
-    cu = w.cu_seqlens.astype(np.int64)
-    if tokens_limit is not None and tokens_limit < w.num_tokens:
-        T = tokens_limit
-        cut = cu[cu < T].tolist() + [T]
-        cu = np.asarray(cut, np.int64)
-    else:
-        T = w.num_tokens
-    tok = w.tokens[:T]
     t0 = time.perf_counter()
-    rows = oracle.rows(tok, cu.astype(np.int32), w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes,
-                       w.offsets, threads=threads)
+    rows = oracle.rows(tok, cu, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes, w.offsets,
+                       threads=threads)
     if w.table_dtype == 2:
-        oracle.gather_e4m3(rows, table_host)
+        oracle.gather_e4m3(rows_c, table_c)
     else:
-        oracle.gather(rows, table_host, threads=threads)
-    oracle.grad_sums(rows, grad_host[: rows.size], threads=threads)
-    return T, time.perf_counter() - t0
+        oracle.gather(rows_c, table_c, threads=threads)
+    if grad_host is not None:
+        oracle.grad_sums(rows, grad_host, threads=threads)
+    return time.perf_counter() - t0
+
+
+def sample_prefix(w, tokens_limit):
+    """The first tokens_limit tokens (whole sequences cut at that point)."""
+    cu = w.cu_seqlens.astype(np.int64)
+    if tokens_limit is None or tokens_limit >= w.num_tokens:
+        return w.tokens, w.cu_seqlens.astype(np.int32)
+    T = tokens_limit
+    return w.tokens[:T], np.asarray(cu[cu < T].tolist() + [T], np.int32)
+
+
+def oracle_inputs(w, tok, cu, with_grad, table_rows=None):
+    """Host inputs of one oracle pass over (tok, cu): compact table, rows
+    renumbered into it, and the grad_out rows (bookkeeping, untimed)."""
+    import oracle
+    import synth
+
+    rows = oracle.rows(tok, cu, w.ngram_size, w.heads_per_ngram, w.eos_id, w.mults, w.primes, w.offsets)
+    table_c, rows_c = compact_table(w, rows, table_rows or w.table_rows)
+    grad = None
+    if with_grad:
+        grad = synth.dense_values(w.grad_seed, rows.size * w.head_dim, w.grad_sigma,
+                                  w.grad_dtype).reshape(rows.size, w.head_dim)
+    return table_c, rows_c, grad
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the CPU oracle on bounded samples of the workload."""
+    """--impl reference: the CPU oracle on bounded samples of the workload
+    (the first --ref-tokens tokens of every part of the step)."""
     if rank != 0:
         return 0
-    import synth
-
-    w = workload(args.workload, args.seed)
     threads = os.cpu_count() or 1
-    sample = min(w.num_tokens, args.ref_tokens)
-    # host copies of the inputs the sample touches (table rows regenerated on the host)
-    import oracle
+    parts = []
+    for name, bwd in step_parts(args):
+        w = workload(name, args.seed)
+        tok, cu = sample_prefix(w, args.ref_tokens)
+        parts.append((w, tok, cu) + oracle_inputs(w, tok, cu, bwd))
 
-    rows_s = oracle.rows(w.tokens[:sample], np.asarray([0] + [c for c in w.cu_seqlens[1:] if c < sample] + [sample],
-                                                         np.int32), w.ngram_size, w.heads_per_ngram, w.eos_id,
-                         w.mults, w.primes, w.offsets)
-    # a full-size host table whose touched rows hold the generated values
-    # (np.zeros pages stay unbacked until written, so untouched rows cost no RAM)
-    table_host = np.zeros((w.num_rows, w.head_dim), HOST_DTYPE[w.table_dtype])
-    uniq = np.unique(rows_s)
-    table_host[uniq] = w.table_rows(uniq)
-    grad_host = synth.dense_values(w.grad_seed, rows_s.size * w.head_dim, w.grad_sigma,
-                                   w.grad_dtype).reshape(rows_s.size, w.head_dim)
+    def one_step():
+        return sum(cpu_oracle_pass(w, tok, cu, tc, rc, g, threads) for w, tok, cu, tc, rc, g in parts)
+
     for _ in range(args.warmup):
-        cpu_oracle_step(w, table_host, grad_host, threads, sample)
-    times = []
-    for _ in range(args.steps):
-        T, dt = cpu_oracle_step(w, table_host, grad_host, threads, sample)
-        times.append(dt)
+        one_step()
+    times = [one_step() for _ in range(args.steps)]
+    T = sum(len(p[1]) for p in parts)
     ms = 1e3 * sum(times) / len(times)
     value = T / (ms / 1e3)
+    what = "; ".join(f"{p[0].name}: first {len(p[1])} of {p[0].num_tokens} tokens (rows, gather"
+                     f"{', grad sums' if p[5] is not None else ''})" for p in parts)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int64+f32", "data": "synthetic",
-            "config": describe(w),
+            "config": config_of([p[0] for p in parts], step_parts(args)),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"first {T} of {w.num_tokens} tokens per step (rows, gather, grad sums)"},
+                             "sample": what + " per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def config_of(ws, parts):
+    if len(ws) == 1:
+        return describe(ws[0])
+    return {"workload": " + ".join(f"{w.name} ({'fwd+bwd' if bwd else 'fwd'})" for w, (_, bwd) in zip(ws, parts)),
+            "parts": [dict(describe(w), timed="ple_lookup + ple_grad_scatter" if bwd else "ple_lookup")
+                      for w, (_, bwd) in zip(ws, parts)]}
+
+
+class Part:
+    """Device state of one workload of the step: table, tokens, outputs and,
+    with a backward, grad_out, table_grad and the gradient workspace."""
+
+    def __init__(self, name, do_bwd, seed, dev, sl=None):
+        import torch
+
+        import hashed_gram_embedding_ple_b200 as ple
+        from synth import gpu as sgpu
+
+        self.ple = ple
+        self.w = w = workload(name, seed)
+        self.do_bwd = do_bwd
+        self.sl = sl
+        self.plan = ple.Plan.from_workload(w)
+        T, H, D = w.num_tokens, w.num_heads, w.head_dim
+        tdt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float8_e4m3fn}[w.table_dtype]
+        self.table = torch.empty(w.num_rows, D, dtype=tdt, device=dev)
+        sgpu.fill_(self.table, w.table_seed, w.table_sigma)
+        self.tokens = torch.from_numpy(w.tokens).to(dev)
+        self.cu = torch.from_numpy(w.cu_seqlens).to(dev)
+        self.T_out = T if sl is None else (T // sl[0]) * (sl[2] - sl[1])  # tokens looked up per step
+        self.out = torch.empty(self.T_out, H, D, dtype=self.plan.out_dtype, device=dev)
+        self.rows = torch.empty(self.T_out, H, dtype=torch.int64, device=dev)
+        self.grad = self.table_grad = self.ws = None
+        if do_bwd:
+            gdt = torch.bfloat16 if w.grad_dtype == 1 else torch.float32
+            self.grad = torch.empty(self.T_out * H, D, dtype=gdt, device=dev)
+            sgpu.fill_(self.grad, w.grad_seed, w.grad_sigma)
+            self.table_grad = torch.zeros(w.num_rows, D, dtype=torch.float32, device=dev)
+            self.ws = ple.alloc_workspace(self.plan, self.T_out * H, dev)
+        self.U = None
+
+    def lookup(self, tok=None, cu=None):
+        tok = self.tokens if tok is None else tok
+        cu = self.cu if cu is None else cu
+        sl, T, H, D = self.sl, self.w.num_tokens, self.w.num_heads, self.w.head_dim
+        if sl is None:
+            self.ple.ple_lookup(self.plan, tok, cu, self.table, out=self.out, rows_out=self.rows)
+        else:
+            self.ple.ple_lookup_slice(self.plan, tok, cu, sl[0], sl[1], sl[2], self.table,
+                                      out=self.out.view(T // sl[0], sl[2] - sl[1], H, D),
+                                      rows_out=self.rows.view(T // sl[0], sl[2] - sl[1], H))
+
+    def backward(self, grad=None):
+        self.ple.ple_grad_scatter(self.plan, self.rows.view(-1), self.grad if grad is None else grad, self.table_grad,
+                                  workspace=self.ws)
+
+    def launches(self):
+        """Kernels per step: the lookup; the backward's clear, key_hist, one
+        sort pass per 8-bit digit of the row ids, and the fold."""
+        passes = max(1, (int(self.w.num_rows).bit_length() + 7) // 8)
+        return 1 + (3 + passes if self.do_bwd else 0)
+
+    def fwd_bytes(self):
+        w = self.w
+        N_out = self.T_out * w.num_heads
+        return 8 * w.num_tokens + N_out * w.head_dim * (ELEM_BYTES[w.table_dtype] + self.out.element_size()) + 8 * N_out
+
+    def bwd_bytes(self):
+        w = self.w
+        N = self.T_out * w.num_heads
+        e_g = 2 if w.grad_dtype == 1 else 4
+        return 8 * N + N * w.head_dim * e_g + 2 * self.U * w.head_dim * 4
+
+
+LOOKUP_SRC = ["hashed_gram_embedding_ple_b200/csrc/lookup.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+GRAD_SRC = ["hashed_gram_embedding_ple_b200/csrc/grad.cu", "hashed_gram_embedding_ple_b200/csrc/sort.cuh",
+            "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
 
 
 def main():
@@ -250,14 +368,16 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="single_layer_bf16")
+    ap.add_argument("--workload", default="headline",
+                    help="'headline' (large_table fwd + backward_stress fwd+bwd), a workload name, or "
+                         "sweep:key=value,...")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--fwd-only", action="store_true", help="time the lookup alone (workloads marked fwd only)")
+    ap.add_argument("--fwd-only", action="store_true", help="time the lookup alone (single workload)")
     ap.add_argument("--slice", default=None, metavar="ROW_LEN:START:END",
                     help="time the global-slice lookup of [START, END) of every ROW_LEN-token row (fwd only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--ref-tokens", type=int, default=32768)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--conv", action="store_true",
                     help="time the PLE layer's short convolution (forward + backward) instead of the lookup")
@@ -268,6 +388,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.workload == "headline" and (args.fwd_only or args.slice or args.host_table):
+        raise SystemExit("--fwd-only, --slice and --host-table need a single --workload")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -278,8 +400,6 @@ def main():
     import torch
 
     import hashed_gram_embedding_ple_b200 as ple
-    import synth
-    from synth import gpu as sgpu
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
@@ -298,42 +418,21 @@ def main():
         return run_conv(args, rank, world, dev, dist)
     if args.host_table:
         return run_host_table(args, rank, world, dev, dist)
-    w = workload(args.workload, replica_seed(args.seed, rank))
-    plan = ple.Plan.from_workload(w)
-    T, H, D, N = w.num_tokens, w.num_heads, w.head_dim, w.num_hits
     sl = None
     if args.slice:
         row_len, s0, s1 = (int(x) for x in args.slice.split(":"))
-        if row_len < 1 or T % row_len or not (0 <= s0 < s1 <= row_len):
-            raise SystemExit("--slice needs ROW_LEN dividing the tokens and 0 <= START < END <= ROW_LEN")
         sl = (row_len, s0, s1)
         args.fwd_only = True
-    tdt = {0: torch.float32, 1: torch.bfloat16, 2: torch.float8_e4m3fn}[w.table_dtype]
-    odt = plan.out_dtype  # bf16 for an fp8 table
-    gdt = torch.bfloat16 if w.grad_dtype == 1 else torch.float32
-    log(f"[rank {rank}] workload {w.name}: T={T} H={H} D={D} rows={w.num_rows} table {w.table_bytes / 1e9:.2f} GB")
-
-    table = torch.empty(w.num_rows, D, dtype=tdt, device=dev)
-    sgpu.fill_(table, w.table_seed, w.table_sigma)
-    tokens = torch.from_numpy(w.tokens).to(dev)
-    cu = torch.from_numpy(w.cu_seqlens).to(dev)
-    T_out = T if sl is None else (T // sl[0]) * (sl[2] - sl[1])  # tokens looked up per step
-    out = torch.empty(T_out, H, D, dtype=odt, device=dev)
-    rows = torch.empty(T_out, H, dtype=torch.int64, device=dev)
-
-    def lookup(tok_in, cu_in):
-        if sl is None:
-            ple.ple_lookup(plan, tok_in, cu_in, table, out=out, rows_out=rows)
-        else:
-            ple.ple_lookup_slice(plan, tok_in, cu_in, sl[0], sl[1], sl[2], table,
-                                 out=out.view(T // sl[0], sl[2] - sl[1], H, D),
-                                 rows_out=rows.view(T // sl[0], sl[2] - sl[1], H))
-    do_bwd = not args.fwd_only
-    if do_bwd:
-        grad = torch.empty(N, D, dtype=gdt, device=dev)
-        sgpu.fill_(grad, w.grad_seed, w.grad_sigma)
-        table_grad = torch.zeros(w.num_rows, D, dtype=torch.float32, device=dev)
-        ws = ple.alloc_workspace(plan, N, dev)
+    spec = step_parts(args)
+    parts = []
+    for name, bwd in spec:
+        p = Part(name, bwd, replica_seed(args.seed, rank), dev, sl)
+        if sl is not None and (sl[0] < 1 or p.w.num_tokens % sl[0] or not (0 <= sl[1] < sl[2] <= sl[0])):
+            raise SystemExit("--slice needs ROW_LEN dividing the tokens and 0 <= START < END <= ROW_LEN")
+        w = p.w
+        log(f"[rank {rank}] {w.name}{' (fwd+bwd)' if bwd else ' (fwd)'}: T={w.num_tokens} H={w.num_heads} "
+            f"D={w.head_dim} rows={w.num_rows} table {w.table_bytes / 1e9:.2f} GB")
+        parts.append(p)
     flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -342,15 +441,26 @@ def main():
         flush_w.zero_()
         flush_r.sum()
 
-    def step():
-        lookup(tokens, cu)
-        if do_bwd:
-            ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
+    def step(evs=None):
+        k = 0
+        if evs is not None:
+            evs[k].record(stream)
+        for p in parts:
+            p.lookup()
+            k += 1
+            if evs is not None:
+                evs[k].record(stream)
+            if p.do_bwd:
+                p.backward()
+                k += 1
+                if evs is not None:
+                    evs[k].record(stream)
 
     # unique rows for the backward's algorithmic bytes (bookkeeping, untimed)
     step()
     torch.cuda.synchronize()
-    U = int(torch.unique(rows).numel())
+    for p in parts:
+        p.U = int(torch.unique(p.rows).numel())
     status = ple.ple_status(dev)
     if status != ple.PLE_OK:
         raise SystemExit(f"libple async status {status}")
@@ -360,7 +470,8 @@ def main():
         step()
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    n_ev = 1 + sum(1 + p.do_bwd for p in parts)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
     sampler.start()
     time.sleep(0.3)
@@ -370,12 +481,7 @@ def main():
     wall0 = time.perf_counter()
     for k in range(args.steps):
         flush_l2()                         # L2 flush between steps, outside the events
-        ev[k][0].record(stream)
-        lookup(tokens, cu)
-        ev[k][1].record(stream)
-        if do_bwd:
-            ple.ple_grad_scatter(plan, rows.view(-1), grad, table_grad, workspace=ws)
-        ev[k][2].record(stream)
+        step(ev[k])
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -385,135 +491,174 @@ def main():
     if status != ple.PLE_OK:
         raise SystemExit(f"libple async status {status}")
 
-    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)]
-    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)]
-    step_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)] if do_bwd else list(fwd_ms)
-    ms_step, ms_fwd, ms_bwd = reduce_max([statistics.mean(step_ms), statistics.mean(fwd_ms),
-                                          statistics.mean(bwd_ms)], dist, dev)
+    # per part: mean forward and backward times over the steps, max over ranks
+    means, k = [], 0
+    for p in parts:
+        f = statistics.mean(ev[s][k].elapsed_time(ev[s][k + 1]) for s in range(args.steps))
+        k += 1
+        b = None
+        if p.do_bwd:
+            b = statistics.mean(ev[s][k].elapsed_time(ev[s][k + 1]) for s in range(args.steps))
+            k += 1
+        means += [f, b if b is not None else 0.0]
+    ms_step = statistics.mean(ev[s][0].elapsed_time(ev[s][n_ev - 1]) for s in range(args.steps))
+    red = reduce_max(means + [ms_step], dist, dev)
+    ms_step = red[-1]
+    for i, p in enumerate(parts):
+        p.ms_fwd = red[2 * i]
+        p.ms_bwd = red[2 * i + 1] if p.do_bwd else None
 
     peak, peak_kind = measured_peaks()
-    e_t = ELEM_BYTES[w.table_dtype]
-    e_o = out.element_size()
-    e_g = 2 if w.grad_dtype == 1 else 4
-    N_out = T_out * H
-    fwd_bytes = 8 * T + N_out * D * (e_t + e_o) + 8 * N_out
-    bwd_bytes = 8 * N + N * D * e_g + 2 * U * D * 4
-    fwd_gbs = fwd_bytes / (ms_fwd * 1e-3) / 1e9
-    bwd_gbs = bwd_bytes / (ms_bwd * 1e-3) / 1e9 if do_bwd else None
+    fwd_part = parts[0]
+    bwd_part = next((p for p in parts if p.do_bwd), None)
 
-    # roofline of the dominant call of the step
-    lookup_src = ["hashed_gram_embedding_ple_b200/csrc/lookup.cu", "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
-    grad_src = ["hashed_gram_embedding_ple_b200/csrc/grad.cu", "hashed_gram_embedding_ple_b200/csrc/sort.cuh",
-                "hashed_gram_embedding_ple_b200/csrc/common.cuh"]
+    def part_line(p):
+        fb = p.fwd_bytes()
+        d = {"workload": p.w.name, "fwd": {"ms": p.ms_fwd, "tokens_per_s": world * p.T_out / (p.ms_fwd * 1e-3),
+                                           "gb_per_s": fb / (p.ms_fwd * 1e-3) / 1e9,
+                                           "frac_of_8tbs": fb / (p.ms_fwd * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+                                           "frac_of_measured": fb / (p.ms_fwd * 1e-3) / 1e9 / peak,
+                                           "algorithmic_bytes": fb}}
+        if p.do_bwd:
+            bb = p.bwd_bytes()
+            d["bwd"] = {"ms": p.ms_bwd, "tokens_per_s": world * p.T_out / (p.ms_bwd * 1e-3),
+                        "gb_per_s": bb / (p.ms_bwd * 1e-3) / 1e9,
+                        "frac_of_8tbs": bb / (p.ms_bwd * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+                        "frac_of_measured": bb / (p.ms_bwd * 1e-3) / 1e9 / peak,
+                        "algorithmic_bytes": bb, "unique_rows": p.U}
+        return d
+
+    fwd_bytes = fwd_part.fwd_bytes()
+    fwd_gbs = fwd_bytes / (fwd_part.ms_fwd * 1e-3) / 1e9
     copy_gbs = size_matched_copy_gbs(fwd_bytes, flush_l2, stream, dev)
     fwd_roof = {"bound": "hbm", "achieved": fwd_gbs, "peak": peak, "unit": "GB/s", "frac": fwd_gbs / peak,
                 "size_matched_copy": {"gb_per_s": copy_gbs, "frac": fwd_gbs / copy_gbs,
                                       "what": "torch device copy of the lookup's algorithmic bytes (half read, "
                                               "half written), L2 flushed, CUDA events, outside the timed steps"},
                 "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": fwd_bytes,
-                "traffic": traffic_from_profiles(f"lookup_{w.name}", lookup_src), "kernel": "lookup_kernel",
+                "workload": fwd_part.w.name,
+                "traffic": traffic_from_profiles(f"lookup_{fwd_part.w.name}", LOOKUP_SRC), "kernel": "lookup_kernel",
                 "peak_source": f"{peak_kind} hbm_gbs"}
     roofline = fwd_roof
     bwd_roof = None
-    if do_bwd:
+    if bwd_part is not None:
+        bwd_bytes = bwd_part.bwd_bytes()
+        bwd_gbs = bwd_bytes / (bwd_part.ms_bwd * 1e-3) / 1e9
         bwd_roof = {"bound": "hbm", "achieved": bwd_gbs, "peak": peak, "unit": "GB/s", "frac": bwd_gbs / peak,
                     "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": bwd_bytes,
-                    "traffic": traffic_from_profiles(f"grad_scatter_{w.name}", grad_src),
-                    "kernel": "ple_grad_scatter (sort + fold kernels)", "unique_rows": U,
+                    "workload": bwd_part.w.name,
+                    "traffic": traffic_from_profiles(f"grad_scatter_{bwd_part.w.name}", GRAD_SRC),
+                    "kernel": "ple_grad_scatter (sort + fold kernels)", "unique_rows": bwd_part.U,
                     "peak_source": f"{peak_kind} hbm_gbs"}
-        if ms_bwd > ms_fwd:
+        if bwd_part.ms_bwd > fwd_part.ms_fwd:
             roofline = bwd_roof
 
-    # lookup_kernel; the backward: clear, key_hist, one sort_pass per 8-bit digit of the row ids, the fold
-    sort_passes = max(1, (int(w.num_rows).bit_length() + 7) // 8)
-    launches_per_step = 1 + (3 + sort_passes if do_bwd else 0)
-    value = world * T_out / (ms_step * 1e-3)
+    tokens_per_step = sum(p.T_out for p in parts)
+    value = world * tokens_per_step / (ms_step * 1e-3)
 
     # end to end through the public API with host buffers
     e2e = None
     if args.e2e_steps > 0:
-        h_tok = torch.from_numpy(w.tokens).pin_memory()
-        h_cu = torch.from_numpy(w.cu_seqlens).pin_memory()
-        h_out = torch.empty(T_out, H, D, dtype=odt).pin_memory()
-        h_grad = grad.cpu().pin_memory() if do_bwd else None
+        for p in parts:
+            p.h_tok = torch.from_numpy(p.w.tokens).pin_memory()
+            p.h_cu = torch.from_numpy(p.w.cu_seqlens).pin_memory()
+            p.h_out = torch.empty_like(p.out, device="cpu").pin_memory()
+            p.h_grad = p.grad.cpu().pin_memory() if p.do_bwd else None
+            p.d_tok, p.d_cu = torch.empty_like(p.tokens), torch.empty_like(p.cu)
+            p.d_grad = torch.empty_like(p.grad) if p.do_bwd else None
+            p.ev_fwd, p.ev_up = torch.cuda.Event(), torch.cuda.Event()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d_tok, d_cu = torch.empty_like(tokens), torch.empty_like(cu)
-        d_grad = torch.empty_like(grad) if do_bwd else None
         # the link is full duplex: grad_out goes up on one copy stream from the
-        # step's start, the lookup output comes down on another as soon as the
-        # lookup is done, while the backward runs on the compute stream
+        # step's start, each lookup output comes down on another as soon as
+        # its lookup is done, while the compute stream runs the next call
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev_start, ev_fwd, ev_up, ev_down = (torch.cuda.Event() for _ in range(4))
+        ev_start, ev_down = torch.cuda.Event(), torch.cuda.Event()
         times = []
         for k in range(args.e2e_steps + 2):
             flush_l2()
             e0.record(stream)
             ev_start.record(stream)
-            if do_bwd:
-                up.wait_event(ev_start)
-                with torch.cuda.stream(up):
-                    d_grad.copy_(h_grad, non_blocking=True)
-                    ev_up.record(up)
-            d_tok.copy_(h_tok, non_blocking=True)
-            d_cu.copy_(h_cu, non_blocking=True)
-            lookup(d_tok, d_cu)
-            ev_fwd.record(stream)
-            down.wait_event(ev_fwd)
-            with torch.cuda.stream(down):
-                h_out.copy_(out, non_blocking=True)
-                ev_down.record(down)
-            if do_bwd:
-                stream.wait_event(ev_up)
-                ple.ple_grad_scatter(plan, rows.view(-1), d_grad, table_grad, workspace=ws)
+            up.wait_event(ev_start)
+            with torch.cuda.stream(up):
+                for p in parts:
+                    if p.do_bwd:
+                        p.d_grad.copy_(p.h_grad, non_blocking=True)
+                        p.ev_up.record(up)
+            for p in parts:
+                p.d_tok.copy_(p.h_tok, non_blocking=True)
+                p.d_cu.copy_(p.h_cu, non_blocking=True)
+                p.lookup(p.d_tok, p.d_cu)
+                p.ev_fwd.record(stream)
+                down.wait_event(p.ev_fwd)
+                with torch.cuda.stream(down):
+                    p.h_out.copy_(p.out, non_blocking=True)
+                if p.do_bwd:
+                    stream.wait_event(p.ev_up)
+                    p.backward(p.d_grad)
+            ev_down.record(down)
             stream.wait_event(ev_down)
             e1.record(stream)
             torch.cuda.synchronize()
             if k >= 2:
                 times.append(e0.elapsed_time(e1))
         (t_e2e_ms,) = reduce_max([statistics.mean(times)], dist, dev)
-        h2d = 8 * T + 4 * (len(w.cu_seqlens)) + (N * D * e_g if do_bwd else 0)
-        e2e = {"value": world * T / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": N_out * D * e_o, "ms_per_step": t_e2e_ms,
-               "what": "pinned H2D tokens+cu_seqlens, ple_lookup, D2H of the lookup output; H2D of grad_out on a "
-                       "second copy stream from the step's start, then ple_grad_scatter; the D2H on a third stream "
-                       "beside it (full-duplex link); all inside the CUDA events"}
+        h2d = sum(8 * p.w.num_tokens + 4 * len(p.w.cu_seqlens) + (p.grad.numel() * p.grad.element_size()
+                                                                     if p.do_bwd else 0) for p in parts)
+        d2h = sum(p.out.numel() * p.out.element_size() for p in parts)
+        e2e = {"value": world * tokens_per_step / (t_e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e_ms,
+               "what": "per part: pinned H2D tokens+cu_seqlens, ple_lookup, D2H of the lookup output on a second "
+                       "copy stream; H2D of grad_out on a third stream from the step's start, then "
+                       "ple_grad_scatter (full-duplex link); all inside the CUDA events"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and sl is None:
         threads = os.cpu_count() or 1
-        uniq_rows = torch.unique(rows)
-        table_host = np.zeros((w.num_rows, D), HOST_DTYPE[w.table_dtype])
-        raw = table.view(torch.uint8) if w.table_dtype == 2 else table
-        table_host[uniq_rows.cpu().numpy()] = torch_to_np(raw.index_select(0, uniq_rows))
-        grad_host = torch_to_np(grad) if do_bwd else np.zeros((N, D), np.float32)
+        inputs = []
+        for p in parts:
+            raw = p.table.view(torch.uint8) if p.w.table_dtype == 2 else p.table
+
+            def from_device(uniq, raw=raw):  # the device table's rows (exactly the generator's values)
+                idx = torch.from_numpy(uniq).to(dev)
+                return torch_to_np(raw.index_select(0, idx))
+
+            tc, rc, _ = oracle_inputs(p.w, p.w.tokens, p.w.cu_seqlens, False, from_device)
+            g = torch_to_np(p.grad) if p.do_bwd else None
+            inputs.append((p.w, p.w.tokens, p.w.cu_seqlens, tc, rc, g))
         tot_t, tot_s, reps = 0, 0.0, 0
         while tot_s < args.cpu_seconds and reps < 500:
-            tt, dt = cpu_oracle_step(w, table_host, grad_host, threads)
-            tot_t += tt
-            tot_s += dt
+            for w, tok, cu, tc, rc, g in inputs:
+                tot_s += cpu_oracle_pass(w, tok, cu, tc, rc, g, threads)
+                tot_t += len(tok)
             reps += 1
         cpu = {"value": tot_t / tot_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{reps} full passes of the workload ({T} tokens each): rows, gather, gradient sums; "
+               "sample": f"{reps} full passes of the step's workloads ({tokens_per_step} tokens each): rows, gather "
+                         f"(from a host table of the touched rows), gradient sums for the backward part; "
                          f"std::thread over sequences / hits / rows, {tot_s:.1f} s"}
-        del table_host
+        del inputs
 
     if rank == 0:
+        single = len(parts) == 1
+        w0 = parts[0].w
+        step_desc = " + ".join(("ple_lookup (rows saved) + ple_grad_scatter" if p.do_bwd else "ple_lookup")
+                               + ("" if single else f" on {p.w.name}") for p in parts)
+        if sl is not None:
+            step_desc = f"ple_lookup_slice rows of {sl[0]}, positions [{sl[1]}, {sl[2]})"
+        fl = part_line(fwd_part)["fwd"]
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": ("int64 hash, e4m3->bf16 widening copy, f32 grad" if w.table_dtype == 2 else
-                          f"int64 hash, {DTYPE_NAMES[w.table_dtype]} copy, f32 grad"), "data": "synthetic",
-                "config": dict(describe(w), parallelism=f"replicas{world}",
-                               l2="flushed between steps (512 MB written, then another 512 MB read); flush outside the step events",
-                               step=("ple_lookup (rows saved) + ple_grad_scatter" if do_bwd else
-                                     "ple_lookup" if sl is None else
-                                     f"ple_lookup_slice rows of {sl[0]}, positions [{sl[1]}, {sl[2]})")),
-                "fwd": {"ms": ms_fwd, "tokens_per_s": world * T_out / (ms_fwd * 1e-3), "gb_per_s": fwd_gbs,
-                        "frac_of_8tbs": fwd_gbs / NOMINAL_HBM_GBS, "frac_of_measured": fwd_gbs / peak},
-                "bwd": None if not do_bwd else {
-                    "ms": ms_bwd, "tokens_per_s": world * T / (ms_bwd * 1e-3), "gb_per_s": bwd_gbs,
-                    "frac_of_8tbs": bwd_gbs / NOMINAL_HBM_GBS, "frac_of_measured": bwd_gbs / peak},
+                "vs_baseline": None,
+                "dtype": ("int64 hash, e4m3->bf16 widening copy, f32 grad" if w0.table_dtype == 2 else
+                          f"int64 hash, {DTYPE_NAMES[w0.table_dtype]} copy, f32 grad"), "data": "synthetic",
+                "config": dict(config_of([p.w for p in parts], spec), parallelism=f"replicas{world}",
+                               l2="flushed between steps (512 MB written, then another 512 MB read); flush outside "
+                                  "the step events",
+                               step=step_desc),
+                "fwd": dict(fl, workload=fwd_part.w.name),
+                "bwd": None if bwd_part is None else dict(part_line(bwd_part)["bwd"], workload=bwd_part.w.name),
+                "parts": [part_line(p) for p in parts],
                 "roofline": roofline, "roofline_fwd": fwd_roof, "roofline_bwd": bwd_roof,
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": sum(p.launches() for p in parts) * args.steps,
                 "clocks": clocks, "wall_s_timed_region": wall}
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -17,7 +17,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES]
-    files += [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "sort.cuh"), os.path.join(INCLUDE, "ple.h")]
+    files += [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "sort.cuh"), os.path.join(INCLUDE, "ple.h"),
+              os.path.join(INCLUDE, "ple_debug.h")]
     return files
 
 

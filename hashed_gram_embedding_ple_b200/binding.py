@@ -41,7 +41,9 @@ EXPORTS = ("ple_plan_create", "ple_plan_destroy", "ple_plan_num_heads", "ple_has
            "ple_grad_scatter_noalloc", "ple_grad_scatter_noalloc_scratch_bytes", "ple_prefetch_workspace_bytes",
            "ple_prefetch", "ple_gather_cache", "ple_grad_scatter_cache", "ple_conv_forward",
            "ple_conv_backward_workspace_bytes", "ple_conv_backward", "ple_status", "ple_strerror",
-           "ple_last_cuda_error")
+           "ple_last_cuda_error",
+           # include/ple_debug.h
+           "ple_debug_set_wait_limit_ns", "ple_debug_default_wait_limit_ns")
 
 
 class PleError(RuntimeError):
@@ -99,10 +101,14 @@ def _lib():
         lib.ple_conv_backward_workspace_bytes.restype = sz
         lib.ple_conv_backward.argtypes = [vp, vp, ctypes.c_int, i64, i64, vp, i32, vp, i32, i32, vp, vp, vp, vp, sz,
                                           vp]
-        lib.ple_status.argtypes = [vp]
+        lib.ple_status.argtypes = [vp, vp]
         lib.ple_strerror.argtypes = [ctypes.c_int]
         lib.ple_strerror.restype = ctypes.c_char_p
         lib.ple_last_cuda_error.argtypes = []
+        lib.ple_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.ple_debug_set_wait_limit_ns.restype = ctypes.c_uint64
+        lib.ple_debug_default_wait_limit_ns.argtypes = []
+        lib.ple_debug_default_wait_limit_ns.restype = ctypes.c_uint64
         for name in ("ple_plan_create", "ple_hash", "ple_lookup", "ple_lookup_slice", "ple_gather", "ple_grad_scatter",
                      "ple_grad_prepare", "ple_grad_apply",
                      "ple_grad_scatter_atomic", "ple_grad_scatter_noalloc", "ple_prefetch", "ple_gather_cache",
@@ -487,11 +493,23 @@ def conv_backward(dy, x, cu_seqlens, weight, dilation: int, dx=None, want_dx: bo
     return dx, dweight, dbias
 
 
+def set_wait_limit_ns(ns: int) -> int:
+    """Limit of the bounded waits between blocks for later calls (every
+    device, this process); returns the previous limit (include/ple_debug.h)."""
+    return int(_lib().ple_debug_set_wait_limit_ns(int(ns)))
+
+
+def default_wait_limit_ns() -> int:
+    return int(_lib().ple_debug_default_wait_limit_ns())
+
+
 def noalloc_scratch_bytes() -> int:
     return int(_lib().ple_grad_scatter_noalloc_scratch_bytes())
 
 
-def ple_status(device=None) -> int:
-    """Synchronise the current stream and return (and clear) the async status."""
+def ple_status(device=None, plan: Plan = None) -> int:
+    """Take (return and clear) the async status on the current stream: the
+    word of `plan`, or with no plan every word of the device (all plans and
+    the plan-less calls)."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    return int(_lib().ple_status(_stream(dev)))
+    return int(_lib().ple_status(None if plan is None else plan.handle, _stream(dev)))

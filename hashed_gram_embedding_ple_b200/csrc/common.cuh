@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "ple.h"
@@ -125,13 +126,27 @@ struct ple_plan {
   int32_t head_dim;
   ple_dtype_t table_dtype;
   int32_t row_bytes;
+  int32_t status_slot;  // index of the plan's async status word
+  // per device: the id of the context in which the plan's status word was
+  // last cleared (~0: never)
+  mutable std::atomic<unsigned long long> cleared_ctx[64];
+  ple_plan() : status_slot(0) {
+    for (auto& c : cleared_ctx) c.store(~0ull, std::memory_order_relaxed);
+  }
 };
 
 namespace ple {
-// Device address of the async status word for the current device.
-unsigned int* status_word(cudaError_t* err);
+// Device address of the async status word of `plan` (nullptr: the word of
+// calls that take no plan) on the current device; clears the plan's word on
+// `stream` at its first use in a device context.
+unsigned int* status_word(const ple_plan_t* plan, cudaStream_t stream, cudaError_t* err);
+// The current context's id (false if the driver cannot tell).
+bool current_context_id(unsigned long long* id);
 // Multiprocessor count of the current device (cached).
 int sm_count();
+// Limit, in nanoseconds, of every bounded wait between the blocks of a
+// kernel (the sort's look-back); set by ple_debug_set_wait_limit_ns.
+uint64_t wait_limit_ns();
 // Record a CUDA error for ple_last_cuda_error and return PLE_ERR_CUDA.
 ple_status_t cuda_fail(cudaError_t e);
 // PLE_OK, or cuda_fail of the last launch error.

@@ -592,7 +592,7 @@ ple_status_t ple_conv_forward(const void* x, ple_dtype_t dtype, int64_t T, int64
   if (y == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned16(y) || (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u) != 0)) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(nullptr, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const bool bf = dtype == PLE_BF16;
   const int64_t nvec = C / (bf ? 8 : 4);
@@ -643,7 +643,7 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
     return PLE_OK;  // nothing asked for
   }
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(nullptr, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const bool bf = dtype == PLE_BF16;
   const int64_t nvec = C / (bf ? 8 : 4);

@@ -115,26 +115,105 @@ __device__ __forceinline__ void store_slot(float* __restrict__ base, int64_t slo
   }
 }
 
-// One fp32 reduction per column into table_grad (the single final add).
-template <int CPL>
+// The single final add table_grad[r] + S_r must be the IEEE fp32 add,
+// subnormals included, but the fp32 reductions of global memory
+// (red.global.add.f32 in every vector width, atomicAdd) flush subnormal
+// operands and results to zero on the B200 (checked against IEEE adds on the
+// device).  For |x| >= 2^-100 the two agree: a subnormal table_grad value is
+// then below half an ulp of x and cannot change the rounded sum, and x + t
+// cannot be subnormal unless it is exactly 0 (t and x are then multiples of
+// 2^-124).  So the reduction is used when every value of a lane's group is
+// at least 2^-100 in magnitude (one integer test per group), and any other
+// group (zeros, tiny and subnormal sums, which real gradients almost never
+// produce) is added element by element with an IEEE add:
+//   - by the deterministic folds, as a plain load, add and store: each row's
+//     final add is made once per call, by the lane group that owns the row
+//     (a compare-and-swap loop anywhere in the fold kernel made it about 20 %
+//     slower, even out of line and never executed);
+//   - by the atomic variant, whose hits of one row race, as a
+//     compare-and-swap loop around the add.
+constexpr uint32_t kExactBelow = 0x0D800000u;  // bits of 2^-100
+
+// True if some |v[q]| < 2^-100 (zeros and subnormals included; NaN is not).
+template <int n>
+__device__ __forceinline__ bool any_tiny(const float* v) {
+  uint32_t m = 0xffffffffu;
+#pragma unroll
+  for (int q = 0; q < n; ++q) m = min(m, __float_as_uint(v[q]) & 0x7fffffffu);
+  return m < kExactBelow;
+}
+
+// p += x with an IEEE add; kShared: other threads may add to *p meanwhile.
+template <bool kShared>
+__device__ __forceinline__ void add_exact(float* p, float x) {
+  if constexpr (kShared) {
+    unsigned* q = reinterpret_cast<unsigned*>(p);
+    unsigned old = __ldcg(q);
+    for (;;) {
+      const unsigned want = __float_as_uint(__fadd_rn(__uint_as_float(old), x));
+      const unsigned seen = atomicCAS(q, old, want);
+      if (seen == old) break;
+      old = seen;
+    }
+  } else {
+    __stcg(p, __fadd_rn(__ldcg(p), x));
+  }
+}
+
+__device__ __forceinline__ void red_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <bool kShared>
+__device__ __forceinline__ void red_add1(float* p, float a) {
+  if (any_tiny<1>(&a))
+    add_exact<kShared>(p, a);
+  else
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
+template <bool kShared>
+__device__ __forceinline__ void red_add2(float* p, float a, float b) {
+  const float v[2] = {a, b};
+  if (any_tiny<2>(v)) {
+    add_exact<kShared>(p, a);
+    add_exact<kShared>(p + 1, b);
+  } else {
+    asm volatile("red.global.add.v2.f32 [%0], {%1,%2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+  }
+}
+
+template <bool kShared>
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  const float v[4] = {a, b, c, d};
+  if (any_tiny<4>(v)) {
+    add_exact<kShared>(p, a);
+    add_exact<kShared>(p + 1, b);
+    add_exact<kShared>(p + 2, c);
+    add_exact<kShared>(p + 3, d);
+  } else {
+    red_v4(p, a, b, c, d);
+  }
+}
+
+// One fp32 reduction per column into table_grad (the single final add of a
+// fold, kShared = false; or one hit's add in the atomic variant, kShared).
+template <int CPL, bool kShared>
 __device__ __forceinline__ void red_add_row(float* __restrict__ tg, int64_t row, int D, const Cols<CPL>& x) {
   const int lane = threadIdx.x & 31;
   if constexpr (CPL == 0) {
 #pragma unroll
     for (int k = 0; k < kMaxColsPerLane; ++k)
-      if (lane + 32 * k < D) atomicAdd(tg + row * D + lane + 32 * k, x.v[k]);
+      if (lane + 32 * k < D) red_add1<kShared>(tg + row * D + lane + 32 * k, x.v[k]);
   } else {
     float* p = tg + row * D + lane * CPL;
     if constexpr (CPL == 1) {
-      asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x.v[0]) : "memory");
+      red_add1<kShared>(p, x.v[0]);
     } else if constexpr (CPL == 2) {
-      asm volatile("red.global.add.v2.f32 [%0], {%1,%2};" ::"l"(p), "f"(x.v[0]), "f"(x.v[1]) : "memory");
+      red_add2<kShared>(p, x.v[0], x.v[1]);
     } else {
 #pragma unroll
-      for (int k = 0; k < CPL; k += 4)
-        asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p + k), "f"(x.v[k]), "f"(x.v[k + 1]),
-                     "f"(x.v[k + 2]), "f"(x.v[k + 3])
-                     : "memory");
+      for (int k = 0; k < CPL; k += 4) red_add4<kShared>(p + k, x.v[k], x.v[k + 1], x.v[k + 2], x.v[k + 3]);
     }
   }
 }
@@ -247,8 +326,9 @@ __device__ __forceinline__ bool window_setup(const uint32_t* __restrict__ K, con
 constexpr unsigned kDoneTarget = 1u << 30;
 
 struct RunBook {
-  int* len;        // [windows] run length, written by the last chunk's writer
-  unsigned* done;  // [windows] completion counters, cleared before the fold
+  int* len;               // [windows] run length, written by the last chunk's writer
+  unsigned* done;         // [windows] completion counters, cleared before the fold
+  const uint32_t* abort;  // the sort's abort word: non-zero, the fold writes nothing
 };
 
 __device__ __forceinline__ int64_t chunk_slot(int64_t s, int m) {
@@ -294,10 +374,6 @@ __device__ __forceinline__ int chunk_stored(const Window& W, int c, int nxt, int
   return nc;
 }
 
-__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
 
 // Second level of a long run, by a whole warp after its window is folded:
 // the run's chunk sums go through the warp's staging buffer (`stage_vecs`
@@ -335,7 +411,8 @@ __device__ void finish_run_staged(const float* csum, int64_t s, int nc, int D, u
   for (int j = 0; j < 2; ++j) {
     const int col = lane + 32 * j;
     if (col < vps)
-      red_add4(table_grad + static_cast<int64_t>(key) * D + col * 4, acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      red_add4<false>(table_grad + static_cast<int64_t>(key) * D + col * 4, acc[j][0], acc[j][1], acc[j][2],
+                      acc[j][3]);
   }
 }
 
@@ -430,8 +507,10 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
   wait_for_prior_grid();
   allow_next_grid();
   if (w * 32 >= N) return;
+  const uint32_t aborted = ld_relaxed(rb.abort);  // (in flight with the window's loads)
   Window W;
-  if (!window_setup(K, I, N, w, W)) return;
+  const bool any = window_setup(K, I, N, w, W);
+  if (!any || aborted != 0) return;  // nothing to fold, or the sort gave up: no write at all
   const size_t row_bytes = static_cast<size_t>(D) * (BF16 ? 2 : 4);
   const unsigned char* gbase = static_cast<const unsigned char*>(grad) + sub * 16;
   keys_s[lane] = W.kA;
@@ -451,8 +530,10 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
       const uint64_t later = rem & ~(1ull << r0) & ((2ull << (r0 + kWideRows)) - 1);
       r1 = 63 - __clzll(later);  // a later chunk start within reach exists: chunks are <= 32 long
     }
-    for (int e = r0 + grp; e < r1; e += RPI)
-      cp_async16(rows_s + (e - r0) * L + sub, gbase + static_cast<size_t>(ids_s[e]) * row_bytes);
+    for (int e = r0 + grp; e < r1; e += RPI) {
+      const uint32_t id = ids_s[e];  // < N for a sorted workspace; kept inside grad_out whatever it holds
+      cp_async16(rows_s + (e - r0) * L + sub, gbase + static_cast<size_t>(id < N ? id : 0) * row_bytes);
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
     const uint64_t starts = rem & ((r1 >= 64 ? ~0ull : ((1ull << r1) - 1)));
     rem &= ~starts;
@@ -467,7 +548,7 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
       const bool is_head = (W.hm >> c) & 1ull;
       const bool run_ends = (W.p0 + nxt >= N) || ((W.hm >> nxt) & 1ull);  // nxt < 64 unless the data ends there
       desc_s[lane] = static_cast<uint32_t>(nrel) | (is_head && run_ends ? kChunkWhole : 0u) |
-                     (keys_s[c] == bad_key ? kChunkSkip : 0u);
+                     (keys_s[c] >= bad_key ? kChunkSkip : 0u);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncwarp();
@@ -492,10 +573,13 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
       const uint32_t key = keys_s[c];
       if (dsc & kChunkWhole) {
         float* dst = table_grad + static_cast<int64_t>(key) * D;
+        if (!any_tiny<CPLN>(acc)) {
 #pragma unroll
-        for (int q = 0; q < CPLN; q += 4) {
-          float* d4 = dst + lane_col<L, BF16>(sub, q);
-          red_add4(d4, acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+          for (int q = 0; q < CPLN; q += 4)
+            red_v4(dst + lane_col<L, BF16>(sub, q), acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < CPLN; ++q) add_exact<false>(dst + lane_col<L, BF16>(sub, q & ~3) + (q & 3), acc[q]);
         }
       } else {
         const int nxt = r0 + nrel;
@@ -535,8 +619,10 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
   wait_for_prior_grid();
   allow_next_grid();
   if (w * 32 >= N) return;
+  const uint32_t aborted = ld_relaxed(rb.abort);
   Window W;
-  if (!window_setup(K, I, N, w, W)) return;
+  const bool any = window_setup(K, I, N, w, W);
+  if (!any || aborted != 0) return;
   Cols<0> acc;
 #pragma unroll
   for (int k = 0; k < Cols<0>::n; ++k) acc.v[k] = 0.f;
@@ -548,7 +634,8 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
       const int e = e0 + u;
       if (e < W.b) {
         const uint32_t ia = __shfl_sync(kFull, W.iA, e & 31), ib = __shfl_sync(kFull, W.iB, e & 31);
-        load_cols<0, BF16>(grad, e < 32 ? ia : ib, D, g[u]);
+        const uint32_t id = e < 32 ? ia : ib;
+        load_cols<0, BF16>(grad, id < N ? id : 0, D, g[u]);
       }
     }
 #pragma unroll
@@ -566,10 +653,10 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
         const int nxt = e + 1;
         if (nxt == W.b || ((W.cm >> nxt) & 1ull)) {
           const uint32_t key = W.key_at(c);
-          if (key != bad_key) {
+          if (key < bad_key) {
             int64_t slot = 0;
             if (chunk_is_whole_run(W, c, nxt, N, &slot)) {
-              red_add_row<0>(table_grad, key, D, acc);
+              red_add_row<0, false>(table_grad, key, D, acc);
             } else {
               store_slot<0>(csum, slot, D, acc);
               int64_t s = 0;
@@ -588,7 +675,7 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
                     if (d < D) sum.v[q] = sum.v[q] + __ldcg(csum + chunk_slot(s, m) * D + d);
                   }
                 }
-                red_add_row<0>(table_grad, key, D, sum);
+                red_add_row<0, false>(table_grad, key, D, sum);
               }
             }
           }
@@ -613,7 +700,7 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
     }
     Cols<CPL> x;
     load_cols<CPL, BF16>(grad, i, D, x);
-    red_add_row<CPL>(table_grad, r, D, x);
+    red_add_row<CPL, true>(table_grad, r, D, x);
   }
   if (bad && (threadIdx.x & 31) == 0) raise_flag(status, PLE_ERR_BAD_ROW);
 }
@@ -707,7 +794,7 @@ ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, i
   if (workspace == nullptr || ws_bytes < L.total_bytes) return PLE_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   auto* ws = static_cast<unsigned char*>(workspace);
   const auto s = static_cast<cudaStream_t>(stream);
@@ -715,6 +802,7 @@ ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, i
   RunBook rb;
   rb.len = reinterpret_cast<int*>(ws + L.run_len);
   rb.done = reinterpret_cast<unsigned int*>(ws + L.run_done);
+  rb.abort = sort_abort_word(L.sort, ws);
   const uint32_t* Ks = nullptr;
   const uint32_t* Is = nullptr;
   if (phases & kPrepare) {
@@ -786,7 +874,7 @@ ple_status_t ple_grad_scatter_atomic(const ple_plan_t* plan, const int64_t* rows
   ple_status_t st = check_grad_args(plan, rows, N, grad, gdt, table_grad);
   if (st != PLE_OK || N == 0) return st;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const int D = plan->head_dim;
   const auto s = static_cast<cudaStream_t>(stream);
@@ -832,10 +920,13 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t{32} << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, one per device.  In host code the
-// array's name only stands in for the symbol; its device address has to be
-// looked up with that device current.
+// Device address of g_noalloc_scratch, one per device, with the id of the
+// context it was looked up in.  In host code the array's name only stands in
+// for the symbol; its device address has to be looked up with that device
+// current, and again when the runtime has loaded the module into a new
+// context (after cudaDeviceReset).
 std::atomic<void*> g_noalloc_addr[64];
+std::atomic<unsigned long long> g_noalloc_ctx[64];
 
 }  // namespace
 
@@ -850,10 +941,15 @@ ple_status_t ple_grad_scatter_noalloc(const ple_plan_t* plan, const int64_t* row
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= 64) return PLE_ERR_UNSUPPORTED;
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
   void* scratch = g_noalloc_addr[dev].load(std::memory_order_acquire);
-  if (scratch == nullptr) {  // first call on this device: look the address up
+  if (scratch == nullptr || (have_ctx && g_noalloc_ctx[dev].load(std::memory_order_acquire) != ctx)) {
+    // first call on this device (or in a new context): look the address up
     e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
+    unsigned long long now = 0;
+    if (current_context_id(&now)) g_noalloc_ctx[dev].store(now, std::memory_order_relaxed);
     g_noalloc_addr[dev].store(scratch, std::memory_order_release);
   }
   return ple_grad_scatter(plan, rows, N, grad, gdt, table_grad, scratch, kNoAllocScratchBytes, stream);

@@ -37,13 +37,16 @@ __device__ __forceinline__ unsigned window_heads(const uint32_t* __restrict__ K,
 
 // cnt of every block of kWinWarps windows -> bsum[block]
 __global__ void __launch_bounds__(kWinWarps * 32)
-count_heads_kernel(const uint32_t* __restrict__ K, int64_t N, int64_t nwin, int64_t* __restrict__ bsum) {
+count_heads_kernel(const uint32_t* __restrict__ K, int64_t N, int64_t nwin, int64_t* __restrict__ bsum,
+                   const uint32_t* abort) {
   __shared__ int wsum[kWinWarps];
   wait_for_prior_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWinWarps + warp;
   uint32_t key;
-  const unsigned m = w < nwin ? window_heads(K, N, w, &key) : 0u;
+  // a sort that gave up: no distinct rows (num_unique = 0, nothing copied)
+  const bool stop = ld_relaxed(abort) != 0;
+  const unsigned m = (w < nwin && !stop) ? window_heads(K, N, w, &key) : 0u;
   if (lane == 0) wsum[warp] = __popc(m);
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -95,10 +98,12 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(int64_t* __restrict_
 __global__ void __launch_bounds__(kWinWarps * 32)
 finalize_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, int64_t N, int64_t nwin,
                 const int64_t* __restrict__ bpre, int64_t num_rows, const unsigned char* host_table, int32_t row_bytes,
-                unsigned char* __restrict__ cache, int64_t* __restrict__ slots, int64_t* __restrict__ uniq_rows) {
+                unsigned char* __restrict__ cache, int64_t* __restrict__ slots, int64_t* __restrict__ uniq_rows,
+                const uint32_t* abort) {
   __shared__ int wsum[kWinWarps];
   __shared__ unsigned char head_lane[kWinWarps][32];  // lane of the r-th head of each window
   wait_for_prior_grid();
+  if (ld_relaxed(abort) != 0) return;  // the sort gave up: nothing is written
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWinWarps + warp;
   uint32_t key = 0;
@@ -113,7 +118,10 @@ finalize_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I, 
   unsigned le;
   asm("mov.u32 %0, %%lanemask_le;" : "=r"(le));
   const int64_t u = base + __popc(m & le) - 1;  // distinct rows up to and including p, minus one
-  if (p < N) slots[I[p]] = u;
+  if (p < N) {
+    const uint32_t i = I[p];  // < N for a sorted workspace; no write outside slots whatever it holds
+    if (i < N) slots[i] = u;
+  }
   const bool bad = key >= num_rows;
   if (((m >> lane) & 1u) != 0) uniq_rows[u] = bad ? -1 : static_cast<int64_t>(key);
   // copy the rows of this window's heads: (head h, 16-byte column c) pairs over the lanes
@@ -210,7 +218,7 @@ ple_status_t ple_prefetch(const ple_plan_t* plan, const int64_t* tokens, int64_t
   if (workspace == nullptr || ws_bytes < L.total_bytes) return PLE_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   // rows of every hit (written into slots, overwritten by the slots at the end)
   ple_status_t st = ple_hash(plan, tokens, T, cu, S, slots, stream);
@@ -221,15 +229,16 @@ ple_status_t ple_prefetch(const ple_plan_t* plan, const int64_t* tokens, int64_t
   st = launch_sort(slots, N, plan->num_rows, ws, L.sort, nullptr, 0, status, s, &K, &I);
   if (st != PLE_OK) return st;
   auto* bsum = reinterpret_cast<int64_t*>(ws + L.bsum);
+  const uint32_t* abort = sort_abort_word(L.sort, ws);
   e = launch_after(count_heads_kernel, dim3(static_cast<unsigned>(L.nblocks)), dim3(kWinWarps * 32), 0, s, K, N,
-                   L.nwin, bsum);
+                   L.nwin, bsum, abort);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_after(scan_kernel, dim3(1), dim3(kScanThreads), 0, s, bsum, L.nblocks, num_unique);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_after(finalize_kernel, dim3(static_cast<unsigned>(L.nblocks)), dim3(kWinWarps * 32), 0, s, K, I, N,
                    L.nwin, static_cast<const int64_t*>(bsum), plan->num_rows,
                    static_cast<const unsigned char*>(host_table), plan->row_bytes, static_cast<unsigned char*>(cache),
-                   slots, uniq_rows);
+                   slots, uniq_rows, abort);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }

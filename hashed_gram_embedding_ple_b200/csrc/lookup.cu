@@ -416,7 +416,7 @@ ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t T, 
   if (rows == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(rows, 8)) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const int H = plan->hp.num_heads;
   const size_t smem = H * sizeof(HeadConst) + static_cast<size_t>(kHashWarps) * 32 * H * sizeof(int64_t);
@@ -439,7 +439,7 @@ template <bool kSlice>
 ple_status_t dispatch_lookup(const ple_plan_t* plan, const int64_t* tokens, int64_t T, const int32_t* cu, int32_t S,
                              const void* table, void* out, int64_t* rows_out, const OutMap& om, void* stream) {
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const auto s = static_cast<cudaStream_t>(stream);
   const int64_t Tout = kSlice ? om.count : T;
@@ -474,7 +474,7 @@ ple_status_t gather_bounded(const ple_plan_t* plan, const int64_t* rows, int64_t
   if (rows == nullptr || table == nullptr || out == nullptr) return PLE_ERR_INVALID_ARG;
   if (!aligned(rows, 8) || !aligned(table, 16) || !aligned(out, 16)) return PLE_ERR_ALIGNMENT;
   cudaError_t e;
-  unsigned int* status = status_word(&e);
+  unsigned int* status = status_word(plan, static_cast<cudaStream_t>(stream), &e);
   if (status == nullptr) return cuda_fail(e);
   const dim3 grid(static_cast<unsigned>((N + kGatherHits - 1) / kGatherHits));
   const auto s = static_cast<cudaStream_t>(stream);

@@ -44,9 +44,17 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // A published word is READY | count; the count is the payload, so plain
 // relaxed loads and stores suffice.  Keys then go to digit start + earlier
 // count + rank, written from the staged tile so that the writes are
-// coalesced.  Every wait is bounded: past the limit the block raises
-// PLE_ERR_TIMEOUT and carries on with what it has (the result is then
-// unspecified; nothing hangs).
+// coalesced.
+//
+// Every wait is bounded in time (the device's global nanosecond timer,
+// limit chosen by the host per call).  A warp whose wait runs out raises
+// PLE_ERR_TIMEOUT and sets the call's abort word in the workspace; every
+// other waiting warp sees that word at its next poll and gives up too, later
+// passes return at their first instruction, and the kernels that consume
+// the sort (the gradient's fold, the prefetch's finalize) check the word
+// and write nothing.  A stuck sort thus ends within about one wait limit,
+// leaves its outputs (table_grad, the cache) untouched, and every access on
+// the way stays inside the workspace.
 // ---------------------------------------------------------------------------
 constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
@@ -59,7 +67,6 @@ constexpr int64_t kBigTileKeys = 3 << 17;
 inline int sort_items(int64_t N) { return N >= kBigTileKeys ? 16 : 8; }
 constexpr int kMaxPasses = 4;
 constexpr int kGroupBits = 5;                         // 32 tiles per group, 32 groups per supergroup
-constexpr unsigned kSpinLimit = 1u << 22;             // a few seconds of polling, then give up
 constexpr uint32_t kReady = 0x80000000u;              // look-back word: READY | count (count < 2^31)
 
 // Lanes of the warp holding the same BITS-bit value as this lane (valid
@@ -108,6 +115,26 @@ __device__ __forceinline__ uint4 ld_relaxed_v4(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// What a bounded wait needs: where to raise the error, the call's abort
+// word (cleared at the start of every sort), and the limit in nanoseconds.
+struct WaitCtl {
+  unsigned int* status;
+  uint32_t* abort;
+  uint64_t wait_ns;
+};
+
 __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -123,7 +150,7 @@ __device__ __forceinline__ bool all_ready(const uint4& x) {
 // are loaded again, round after round; the warps' partial sums meet in
 // `part`.  Returns the sum for digit threadIdx.x (threads < 256).
 __device__ uint32_t level_sum(const uint32_t* rows, int64_t first, int64_t last, uint32_t (*part)[kRadix],
-                              unsigned int* status) {
+                              const WaitCtl& wc) {
   if (first >= last) return 0;  // block-uniform
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -139,13 +166,24 @@ __device__ uint32_t level_sum(const uint32_t* rows, int64_t first, int64_t last,
         x[k][0] = x[k][1] = make_uint4(kReady, kReady, kReady, kReady);
       }
     }
-    for (unsigned spins = 0;; ++spins) {
+    uint64_t t0 = 0;
+    for (int round = 0;; ++round) {
       bool ready = true;
 #pragma unroll
       for (int k = 0; k < 4; ++k) ready &= all_ready(x[k][0]) && all_ready(x[k][1]);
       if (__all_sync(kFull, ready)) break;
-      if (spins >= kSpinLimit) {
-        if (lane == 0) raise_flag(status, PLE_ERR_TIMEOUT);
+      // give up when the limit has passed since the first poll, or (looked
+      // at every 16th round, off the common short waits) when another warp
+      // of the call has given up; a warp-uniform decision
+      const uint64_t now = global_ns();
+      if (round == 0) t0 = now;
+      bool give_up = round > 0 && now - t0 >= wc.wait_ns;
+      if ((round & 15) == 15 && lane == 0) give_up |= ld_relaxed(wc.abort) != 0;
+      if (__any_sync(kFull, give_up)) {
+        if (lane == 0) {
+          raise_flag(wc.status, PLE_ERR_TIMEOUT);
+          st_relaxed(wc.abort, 1u);
+        }
         break;
       }
       __nanosleep(64);
@@ -186,7 +224,7 @@ struct SortArgs {
   uint32_t* hist;          // [kMaxPasses][256] digit totals of every pass (zeroed before the sort)
   unsigned int* tickets;   // [kMaxPasses] tile tickets (zeroed before the sort)
   uint32_t* look;          // [passes][tiles + groups + supers][256] published counts
-  unsigned int* status;
+  WaitCtl wc;              // bounded waits; wc.abort is zeroed before the sort with hist and tickets
 };
 
 // Keys from the int64 rows (a row outside [0, num_rows) becomes the key
@@ -232,7 +270,7 @@ key_hist_kernel(const int64_t* __restrict__ rows, int64_t num_rows, const SortAr
       }
     }
   }
-  if (bad) raise_flag(a.status, PLE_ERR_BAD_ROW);
+  if (bad) raise_flag(a.wc.status, PLE_ERR_BAD_ROW);
   __syncthreads();
   for (int k = tid; k < a.passes * kRadix; k += kSortThreads) {
     const uint32_t c = (&h[0][0])[k];
@@ -252,9 +290,13 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   __shared__ uint32_t start_s[kRadix];
   __shared__ uint32_t warp_tot[kSortWarps];
   __shared__ int64_t tile_s;
+  __shared__ uint32_t abort_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   wait_for_prior_grid();
-  if (tid == 0) tile_s = atomicAdd(a.tickets + pass, 1u);
+  if (tid == 0) {
+    abort_s = ld_relaxed(a.wc.abort);  // an earlier wait of this sort gave up: nothing more to do
+    tile_s = atomicAdd(a.tickets + pass, 1u);
+  }
   if (tid < kRadix) start_s[tid] = 0;  // the tile's digit counts first
   {  // global start of every digit of this pass (while the ticket is on its way)
     const uint32_t c = tid < kRadix ? __ldcg(a.hist + pass * kRadix + tid) : 0;
@@ -263,6 +305,7 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
     if (tid < kRadix) base_s[tid] = start;
   }
   allow_next_grid();
+  if (abort_s != 0) return;  // block-uniform (read after the barriers above)
   const int64_t t = tile_s;
   const int64_t N = a.N, i0 = t * kSortTile + warp * kWarpSpan;
   const int shift = 8 * pass;
@@ -293,7 +336,7 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   uint32_t* group_rows = tile_rows + a.tiles * kRadix;
   uint32_t* super_rows = group_rows + a.groups * kRadix;
   const int64_t g = t >> kGroupBits, sg = g >> kGroupBits;
-  uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.status);
+  uint32_t before = level_sum(tile_rows, g << kGroupBits, t, wh, a.wc);
   if ((t & 31) == 31 && tid < kRadix) st_relaxed(group_rows + g * kRadix + tid, kReady | (before + count));
   // then everything local to the tile (its ranks, the tile staged in digit
   // order) while the other groups' totals are published
@@ -338,9 +381,9 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   }
   __syncthreads();
   // keys of digit tid in the earlier groups and supergroups (wh is the scratch again)
-  before += level_sum(group_rows, sg << kGroupBits, g, wh, a.status);
+  before += level_sum(group_rows, sg << kGroupBits, g, wh, a.wc);
   if ((t & 1023) == 1023 && tid < kRadix) st_relaxed(super_rows + sg * kRadix + tid, kReady | (before + count));
-  before += level_sum(super_rows, 0, sg, wh, a.status);
+  before += level_sum(super_rows, 0, sg, wh, a.wc);
   if (tid < kRadix) base_s[tid] += before;
   __syncthreads();
   // coalesced writes: consecutive threads, consecutive destinations within a digit
@@ -387,7 +430,7 @@ inline SortLayout sort_layout(int64_t N, size_t* off) {
   const int64_t small_tiles = (N + kSortThreads * 8 - 1) / (kSortThreads * 8);
   const int64_t small_groups = (small_tiles + 31) >> kGroupBits, small_supers = (small_groups + 31) >> kGroupBits;
   L.look = take(sizeof(uint32_t) * kRadix * kMaxPasses * static_cast<size_t>(small_tiles + small_groups + small_supers));
-  L.zeroed_bytes = sizeof(uint32_t) * (kMaxPasses * kRadix + kMaxPasses);
+  L.zeroed_bytes = sizeof(uint32_t) * (kMaxPasses * kRadix + kMaxPasses + 1);  // totals, tickets, abort word
   L.zeroed = take(L.zeroed_bytes);
   return L;
 }
@@ -397,6 +440,11 @@ inline int sort_passes(int64_t num_rows) {
   int bits = 0;
   while (bits < 32 && (static_cast<uint64_t>(num_rows) >> bits) != 0) ++bits;
   return (bits + 7) / 8 > 1 ? (bits + 7) / 8 : 1;
+}
+
+// The call's abort word (non-zero once a wait of the sort gave up).
+inline uint32_t* sort_abort_word(const SortLayout& L, unsigned char* ws) {
+  return reinterpret_cast<uint32_t*>(ws + L.zeroed) + kMaxPasses * kRadix + kMaxPasses;
 }
 
 // Where the sort leaves its result (keys, values) for keys below num_rows.
@@ -427,7 +475,9 @@ inline ple_status_t launch_sort(const int64_t* rows, int64_t N, int64_t num_rows
   sa.look = reinterpret_cast<uint32_t*>(ws + L.look);
   sa.hist = reinterpret_cast<uint32_t*>(ws + L.zeroed);
   sa.tickets = sa.hist + kMaxPasses * kRadix;
-  sa.status = status;
+  sa.wc.status = status;
+  sa.wc.abort = sort_abort_word(L, ws);
+  sa.wc.wait_ns = wait_limit_ns();
   sa.passes = sort_passes(num_rows);
   cudaError_t e = launch_after(clear_kernel, dim3(1), dim3(kSortThreads), 0, s, sa.hist,
                                static_cast<int>(L.zeroed_bytes / sizeof(uint32_t)));

@@ -34,9 +34,10 @@
  *   - synchronous errors (bad arguments, alignment, workspace size, launch
  *     failure) are returned; nothing is launched when one is returned;
  *   - asynchronous errors found by kernels (a row id outside the table,
- *     malformed cu_seqlens) never trap: the kernel zeroes or skips the
- *     affected output, sets a bit in a per-device status word and carries
- *     on; ple_status reports and clears that word.
+ *     malformed cu_seqlens, a bounded wait that ran out) never trap: the
+ *     kernel zeroes or skips the affected output, sets a bit in the status
+ *     word of the call's plan (on the device it runs on) and carries on;
+ *     ple_status reports and clears that word.
  *   - layouts are dense row-major; int64 rows; tables [num_rows, head_dim].
  */
 #ifndef PLE_H_
@@ -92,9 +93,11 @@ typedef struct ple_plan ple_plan_t;
  * Host only: touches no GPU.  Errors: PLE_ERR_INVALID_ARG (null pointers,
  * ngram_size outside 2..8, heads_per_ngram < 1, a prime < 2 or > 2^62, a
  * negative offset, a head range outside [0, num_rows) or overlapping
- * another), PLE_ERR_UNSUPPORTED (H > 64), PLE_ERR_ALIGNMENT (head_dim *
- * element size not a multiple of 16 bytes).  On success *out owns a plan
- * that ple_plan_destroy frees. */
+ * another), PLE_ERR_UNSUPPORTED (H > 64, or 4095 plans already alive: each
+ * holds one async status word), PLE_ERR_ALIGNMENT (head_dim * element size
+ * not a multiple of 16 bytes).  On success *out owns a plan that
+ * ple_plan_destroy frees; destroy a plan only once its calls have completed
+ * (its status word goes to the next plan created). */
 ple_status_t ple_plan_create(const ple_params_t* params, ple_plan_t** out);
 void ple_plan_destroy(ple_plan_t* plan);
 int32_t ple_plan_num_heads(const ple_plan_t* plan);
@@ -152,8 +155,12 @@ size_t ple_grad_scatter_workspace_bytes(const ple_plan_t* plan, int64_t num_hits
  * add into table_grad.  The result is bit-identical run to run.
  * rows int64 [num_hits]; grad_out [num_hits, head_dim] of grad_dtype;
  * table_grad fp32 [num_rows, head_dim], accumulated into (the caller zeroes
- * it for a fresh gradient).  Hits whose row is outside [0, num_rows) are
- * dropped and raise the async PLE_ERR_BAD_ROW.  table_grad and grad_out
+ * it for a fresh gradient).  Every add is the IEEE fp32 add, subnormals
+ * included (the device's fp32 reductions flush subnormals, so sums below
+ * 2^-100 in magnitude are added by the row's owner with a load and a store):
+ * nothing else may write table_grad while the call runs (two calls that
+ * overlap on the GPU must not share a table_grad).  Hits whose row is
+ * outside [0, num_rows) are dropped and raise the async PLE_ERR_BAD_ROW.  table_grad and grad_out
  * 16-byte aligned; workspace 256-byte aligned.  Errors: PLE_ERR_WORKSPACE,
  * PLE_ERR_UNSUPPORTED (head_dim > 256, num_rows >= 2^32 - 1 or num_hits >= 2^31),
  * PLE_ERR_INVALID_ARG, PLE_ERR_ALIGNMENT, PLE_ERR_CUDA. */
@@ -195,8 +202,9 @@ ple_status_t ple_grad_scatter_atomic(const ple_plan_t* plan, const int64_t* rows
  * process exits.  Sizes whose workspace (ple_grad_scatter_workspace_bytes)
  * exceeds that area are rejected with PLE_ERR_WORKSPACE before anything is
  * launched; use ple_grad_scatter with a caller workspace for them.  The first
- * call on a device looks up the scratch area's device address (make that
- * first call before any stream capture).  All calls share the one area, so
+ * call on a device (and the first after the device's context changed, e.g.
+ * after cudaDeviceReset) looks up the scratch area's device address (make
+ * that first call before any stream capture).  All calls share the one area, so
  * calls that overlap on the GPU (other streams, other host threads) race and
  * must be serialised by the caller; each call clears what must start at zero.
  * Other arguments, errors and results as ple_grad_scatter. */
@@ -302,11 +310,23 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
                                int32_t dilation, void* dx, float* dweight, float* dbias, void* workspace,
                                size_t workspace_bytes, void* stream);
 
-/* Synchronise `stream`, then return and clear the async status word of the
- * current device (PLE_OK if no kernel flagged anything; otherwise the
- * lowest-numbered flagged error).  The word is shared by all plans and
- * streams on the device. */
-ple_status_t ple_status(void* stream);
+/* Async status of the calls made with `plan` on the current device: runs
+ * one small kernel on `stream` that atomically takes (reads and zeroes) the
+ * plan's status word, waits for it, and returns PLE_OK if no kernel of the
+ * plan flagged anything since the last take, otherwise the lowest-numbered
+ * flagged error.  Taken in stream order: flags of kernels queued on
+ * `stream` before the call are included, and a flag that a kernel on
+ * another stream raises while the take runs is either in this result or
+ * left for the next call, never lost (this replaces the pages' device
+ * asserts and symmetric validation).  Each plan has a word of its own (at
+ * most 4095 plans live at once; ple_plan_create returns
+ * PLE_ERR_UNSUPPORTED beyond), so one plan's ple_status leaves the others'
+ * flags alone.  plan == NULL takes every word of the device at once: the
+ * flags of all plans and of the calls that take no plan (the short
+ * convolution).  Synchronises `stream` (the only call that does); not for
+ * use inside a stream capture.  Device addresses are looked up again after
+ * the current context changes (cudaDeviceReset). */
+ple_status_t ple_status(const ple_plan_t* plan, void* stream);
 
 /* Text for a status code (static storage). */
 const char* ple_strerror(ple_status_t status);

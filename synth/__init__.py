@@ -367,6 +367,18 @@ def backward_stress(seed: int = 0, total: int = 131072) -> Workload:
                     offsets, R, 128, DTYPE_BF16, seed + 101, 0.02, DTYPE_BF16, seed + 202, 1.0)
 
 
+def backward_stress_small(seed: int = 0, total: int = 131072) -> Workload:
+    """The backward-stress tokens and hits with 16 primes >= 125,000 (2.0 M
+    rows): a 0.5 GB table and a 1 GB fp32 gradient, for profiler captures of
+    the backward kernels that replay each launch many times."""
+    w = backward_stress(seed, total)
+    rng = np.random.default_rng(seed + 7)
+    mults, primes, offsets, R = _hash_constants(3, 8, 125_000, rng)
+    w.name = "backward_stress_small"
+    w.primes, w.offsets, w.num_rows = primes, offsets, R
+    return w
+
+
 def sweep_point(tokens: int = 131072, head_dim: int = 128, ngram_size: int = 3, heads_per_ngram: int = 8,
                 table_gb: float = 16.0, ids: str = "zipf", seed: int = 0,
                 table_dtype: int = DTYPE_BF16) -> Workload:
@@ -396,4 +408,5 @@ WORKLOADS = {
     "large_table": large_table,
     "backward_stress": backward_stress,
     "large_table_fp8": large_table_fp8,
+    "backward_stress_small": backward_stress_small,
 }

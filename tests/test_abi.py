@@ -14,9 +14,13 @@ from hashed_gram_embedding_ple_b200 import binding
 
 
 def _declared():
-    text = open(os.path.join(ROOT, "include", "ple.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ple_[a-z_]+)\s*\(", text)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(ple_[a-z_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_symbols_exported():
@@ -218,3 +222,29 @@ def test_grad_halves_check_their_own_arguments():
     assert lib.ple_grad_apply(h, 5, 0x2000, 9, 0x3000, 0x4000, need, None) == binding.PLE_ERR_INVALID_ARG
     assert lib.ple_grad_apply(h, 5, 0x2008, 1, 0x3000, 0x4000, need, None) == binding.PLE_ERR_ALIGNMENT
     assert lib.ple_grad_apply(h, 5, 0x2000, 1, 0x3000, 0x4100, need - 256, None) == binding.PLE_ERR_WORKSPACE
+
+
+def test_wait_limit_setter_round_trips():
+    """Host-only hook of include/ple_debug.h: the limit of the bounded waits."""
+    default = ple.default_wait_limit_ns()
+    assert default == 100_000_000
+    prev = ple.set_wait_limit_ns(12345)
+    try:
+        assert prev == default
+        assert ple.set_wait_limit_ns(0) == 12345
+    finally:
+        ple.set_wait_limit_ns(default)
+    assert ple.set_wait_limit_ns(default) == default
+
+
+def test_plans_hold_status_slots_until_destroyed():
+    """Each plan holds one of 4095 status words; destroying plans returns
+    them (host only)."""
+    lib = ple.lib()
+    plans = [_plan() for _ in range(50)]
+    del plans
+    import gc
+
+    gc.collect()
+    many = [_plan() for _ in range(4000)]  # fits only if the 50 above were returned
+    assert len(many) == 4000

@@ -75,7 +75,27 @@ def test_reference_arm_json_line():
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert d["config"]["workload"] == "single_layer_bf16"
+    assert d["config"]["workload"] == "large_table (fwd) + backward_stress (fwd+bwd)"
+    assert [q["workload"] for q in d["config"]["parts"]] == ["large_table", "backward_stress"]
+    assert "first 512 of 65536" in d["cpu_baseline"]["sample"]
+
+
+def test_reference_arm_single_workload():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3",
+                        "--warmup", "3", "--ref-tokens", "512", "--workload", "single_layer_bf16"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["workload"] == "single_layer_bf16" and d["value"] > 0
+
+
+def test_headline_parts():
+    import argparse
+
+    a = argparse.Namespace(workload="headline", fwd_only=False)
+    assert bench.step_parts(a) == [("large_table", False), ("backward_stress", True)]
+    a = argparse.Namespace(workload="tiny", fwd_only=True)
+    assert bench.step_parts(a) == [("tiny", False)]
 
 
 def test_bench_requires_three_warmups():

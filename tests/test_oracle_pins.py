@@ -328,6 +328,34 @@ def test_grad_single_final_add_and_negative_zero():
     assert np.signbit(tg[3, 0])
 
 
+def test_grad_subnormal_sums_exact():
+    """Gradients and prefill that are integer multiples of 2^-149 (fp32
+    subnormals): every partial sum is exact in fp32 (|sum| < 2^-125), so
+    whatever the order the result is the integer sum times 2^-149.  A
+    flush-to-zero add anywhere in the fold would lose them."""
+    rng = np.random.default_rng(8)
+    N, D, R = 700, 4, 9
+    rows = rng.integers(0, R, N)
+    rows[:100] = 2  # one row with a long run (several chunks)
+    k = rng.integers(-1000, 1000, (N, D))
+    m = rng.integers(-1000, 1000, (R, D))
+    g = (k * 2.0 ** -149).astype(np.float32)
+    assert np.all(np.abs(g) < np.float32(2.0 ** -126))
+    tg = (m * 2.0 ** -149).astype(np.float32)
+    oracle.grad_apply(rows, g, tg)
+    want = m.copy()
+    np.add.at(want, rows, k)
+    np.testing.assert_array_equal(tg, (want * 2.0 ** -149).astype(np.float32))
+    # bf16 subnormals: bits S.00000000.MMMMMMM = +-M * 2^-133, sums exact below 2^-109
+    kb = rng.integers(-127, 128, (N, D))
+    bits = (np.where(kb < 0, 0x8000, 0) | np.abs(kb)).astype(np.uint16)
+    tg = np.zeros((R, D), np.float32)
+    oracle.grad_apply(rows, bits, tg)
+    want = np.zeros((R, D), np.int64)
+    np.add.at(want, rows, kb)
+    np.testing.assert_array_equal(tg, (want * 2.0 ** -133).astype(np.float32))
+
+
 def test_grad_rejects_out_of_range():
     with pytest.raises(ValueError):
         oracle.grad_apply(np.array([0, 9]), np.zeros((2, 4), np.float32), np.zeros((5, 4), np.float32))

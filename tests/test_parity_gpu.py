@@ -189,6 +189,63 @@ def test_gradient_both_sort_tile_sizes(cuda_device, N):
     check_backward(w, cuda_device, rows)
 
 
+# fp32 values at the edge of the final add: signed zeros, subnormals, the
+# smallest normal, and values around 2^-100 (the reduction / exact-add switch)
+_SPECIAL_F32 = np.array([0.0, -0.0, 1e-45, -1e-45, 1e-40, -1e-40, 3e-39, -5.877e-39, 2.0 ** -126, -(2.0 ** -127),
+                         2.0 ** -100, -(2.0 ** -101), 1.0, -1.5], np.float32)
+# bf16 bit patterns: +-0, the smallest and largest subnormal, the smallest normal, ordinary values
+_SPECIAL_BF16 = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x807F, 0x0080, 0x8080, 0x0040, 0x3F80, 0xBFC0],
+                         np.uint16)
+
+
+def _special_grad(rng, n, D, gdt, modes):
+    """Per hit row: mode 0 random specials, 1 all -0, 2 all subnormal, 3 all +0."""
+    if gdt == synth.DTYPE_F32:
+        pool, neg0, pos0, sub = _SPECIAL_F32, np.float32(-0.0), np.float32(0.0), _SPECIAL_F32[2:8]
+    else:
+        pool, neg0, pos0, sub = _SPECIAL_BF16, np.uint16(0x8000), np.uint16(0), _SPECIAL_BF16[2:6]
+    g = pool[rng.integers(0, len(pool), (n, D))]
+    g[modes == 1] = neg0
+    g[modes == 3] = pos0
+    g[modes == 2] = sub[rng.integers(0, len(sub), (int((modes == 2).sum()), D))]
+    return g
+
+
+@pytest.mark.parametrize("D,gdt", [(32, synth.DTYPE_F32), (64, synth.DTYPE_BF16), (128, synth.DTYPE_BF16),
+                                   (64, synth.DTYPE_F32), (40, synth.DTYPE_BF16), (200, synth.DTYPE_F32)])
+def test_gradient_signed_zero_and_subnormal(cuda_device, D, gdt):
+    """The final add table_grad + S_r is the IEEE fp32 add: -0 + -0 stays -0,
+    subnormal sums and subnormal prefills are kept.  Rows hit once (whole-run
+    add), 2..33 times, 64, 65 and 1000 times (chunk slots and the run's
+    second level), with all-(-0), all-(+0), all-subnormal and mixed rows, on
+    the wide folds (D = 32, 64, 128) and the generic fold (D = 40, 200)."""
+    dev = cuda_device
+    rng = np.random.default_rng(4000 + D + gdt)
+    counts = [1] * 120 + [2] * 40 + [31, 32, 33] * 6 + [64, 65, 1000]
+    R = len(counts) + 17  # rows never hit keep their prefill
+    rows = np.concatenate([np.full(c, r, np.int64) for r, c in enumerate(counts)])
+    row_mode = rng.integers(0, 4, R)
+    perm = rng.permutation(rows.size)
+    rows = rows[perm]
+    g_host = _special_grad(rng, rows.size, D, gdt, row_mode[rows])
+    prefill = _SPECIAL_F32[rng.integers(0, len(_SPECIAL_F32), (R, D))].copy()
+    prefill[row_mode == 1] = np.float32(-0.0)
+    w = custom_workload("subn", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [R], D, synth.DTYPE_F32, gdt)
+    plan = ple.Plan.from_workload(w)
+    g = values_to_torch(g_host, gdt).to(dev)
+    ref = oracle.grad_apply(rows, g_host, prefill.copy())
+    assert np.any(np.signbit(ref) & (ref == 0)), "the case must hold -0 results"
+    assert np.any((ref != 0) & (np.abs(ref) < np.float32(2.0 ** -126))), "and subnormal results"
+    for entry in ("scatter", "noalloc"):
+        tg = torch.from_numpy(prefill.copy()).to(dev)
+        if entry == "scatter":
+            ple.ple_grad_scatter(plan, dev_i64(rows, dev), g, tg)
+        else:
+            ple.ple_grad_scatter_noalloc(plan, dev_i64(rows, dev), g, tg)
+        assert ple.ple_status() == ple.PLE_OK
+        np.testing.assert_array_equal(tg.cpu().numpy().view(np.uint32), ref.view(np.uint32), err_msg=entry)
+
+
 def test_bad_rows_flagged(cuda_device):
     dev = cuda_device
     w = synth.tiny(0)

@@ -5,9 +5,11 @@ may not call the CUDA allocator, or hot loops where cudaMalloc would
 synchronise the device cannot pass the workspace ple_grad_scatter needs.
 The no-allocation entry point runs the same kernels in a fixed scratch area
 that the library keeps in device memory.  These tests call it through the C
-ABI and hold it to the workspace entry point's result, bit for bit (the
-gradient is deterministic), on two calls in a row with different inputs, so
-that anything a call leaves behind in the shared scratch area would show.
+ABI and hold it to the workspace entry point's result and to the CPU
+oracle, bit for bit (the gradient is deterministic), on calls in a row with
+different inputs, so that anything a call leaves behind in the shared
+scratch area would show.  The last call uses the largest hit count whose
+workspace fits the scratch area (the sort's 4096-key tiles).
 This file is collected last on purpose.
 """
 import ctypes
@@ -16,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import hashed_gram_embedding_ple_b200 as ple
 from hashed_gram_embedding_ple_b200 import binding
@@ -47,19 +50,35 @@ def _inputs(N, D, seed, dev):
                         synth.DTYPE_BF16, seed=seed)
     g = synth.dense_values(w.grad_seed, N * D, 1.0, synth.DTYPE_BF16).reshape(N, D)
     grad = torch.from_numpy(g.view(np.int16)).view(torch.bfloat16).to(dev)
-    return torch.from_numpy(rows).to(dev), grad
+    return rows, g, torch.from_numpy(rows).to(dev), grad
+
+
+def _largest_fitting(plan, cap):
+    lo, hi = 1, 1
+    while ple.workspace_bytes(plan, hi) <= cap:
+        lo, hi = hi, 2 * hi
+    while hi - lo > 1:  # workspace_bytes is non-decreasing in N
+        mid = (lo + hi) // 2
+        if ple.workspace_bytes(plan, mid) <= cap:
+            lo = mid
+        else:
+            hi = mid
+    return lo
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
+def test_noalloc_matches_workspace_entry_point_and_oracle(cuda_device):
     dev = cuda_device
     lib = ple.lib()
     D = 128
     plan = _plan(D)
+    cap = lib.ple_grad_scatter_noalloc_scratch_bytes()
+    n_max = _largest_fitting(plan, cap)
+    assert n_max >= 3 << 17, "the largest fitting size must reach the 4096-key sort tiles"
     stream = torch.cuda.current_stream(dev).cuda_stream
-    for call, (N, seed) in enumerate([(3 * 4096 + 777, 11), (40_000, 12)]):
-        assert ple.workspace_bytes(plan, N) <= lib.ple_grad_scatter_noalloc_scratch_bytes()
-        rows, grad = _inputs(N, D, seed, dev)
+    for call, (N, seed) in enumerate([(3 * 4096 + 777, 11), (40_000, 12), (n_max, 13)]):
+        assert ple.workspace_bytes(plan, N) <= cap
+        rows_np, g_host, rows, grad = _inputs(N, D, seed, dev)
         ref = torch.zeros(70_001, D, device=dev)
         ple.ple_grad_scatter(plan, rows, grad, ref)
         got = torch.zeros(70_001, D, device=dev)
@@ -68,3 +87,6 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
         assert rc == binding.PLE_OK, f"call {call}: status {rc}"
         assert ple.ple_status(dev) == ple.PLE_OK
         assert torch.equal(got.view(torch.int32), ref.view(torch.int32)), f"call {call} differs"
+        want = oracle.grad_apply(rows_np, g_host, np.zeros((70_001, D), np.float32))
+        np.testing.assert_array_equal(got.cpu().numpy().view(np.uint32), want.view(np.uint32),
+                                      err_msg=f"call {call} differs from the oracle")
