@@ -27,8 +27,8 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // key_hist_kernel turns the int64 rows into 32-bit keys and counts the
 // digits of every pass at once, so the global start of each digit is known
 // before the first pass.  Each pass is one sort_pass_kernel launch in which
-// a block takes one tile of consecutive positions (2048 or 4096 keys, by
-// the key count), in the order of a ticket counter (a block only ever waits
+// a block takes one tile of consecutive positions (2048, 4096 or 8192 keys,
+// by the key count), in the order of a ticket counter (a block only ever waits
 // for tiles with lower tickets, whose blocks are already running).  The
 // block counts its keys per digit and publishes the counts at once.  The
 // keys of a digit in all earlier tiles are summed over three levels, so
@@ -39,7 +39,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 //   supergroups before its supergroup (totals published by the last tile of
 //   each supergroup).
 // Between the first level and the other two the block ranks its keys by
-// digit (warp ballots, per-warp running counts: stable) and stages the tile
+// digit (per-warp lane masks per digit, per-warp running counts: stable) and stages the tile
 // in shared memory in digit order, while the other groups publish.
 // A published word is READY | count; the count is the payload, so plain
 // relaxed loads and stores suffice.  Keys then go to digit start + earlier
@@ -58,31 +58,25 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // ---------------------------------------------------------------------------
 constexpr int kSortThreads = 256;
 constexpr int kSortWarps = kSortThreads / 32;
-// Keys per thread: 16 (4096-key tiles, 2 blocks per SM) from kBigTileKeys
-// keys on, else 8 (2048-key tiles, 3 blocks per SM): fewer tiles shorten the
-// look-back, but below about 3 * 2^17 keys there are too few of them to
-// fill the SMs (measured on the B200: 2048-key tiles win at 262144 keys,
-// 4096-key tiles at 524288 and above).
+// Keys per thread: 32 (8192-key tiles, 2 blocks per SM) from kHugeTileKeys
+// keys on, 16 (4096-key tiles, 2 blocks per SM) from kBigTileKeys, else 8
+// (2048-key tiles, 3 blocks per SM): fewer tiles shorten the look-back and
+// the waves of tiles, but below about 3 * 2^17 keys there are too few of
+// them to fill the SMs (measured on the B200: 2048-key tiles win at 262144
+// keys, 4096-key tiles at 524288; at 2097152 keys 8192-key tiles take a
+// pass from two waves to one, 286.7 -> 276.5 us for the whole gradient).
 constexpr int64_t kBigTileKeys = 3 << 17;
-inline int sort_items(int64_t N) { return N >= kBigTileKeys ? 16 : 8; }
+constexpr int64_t kHugeTileKeys = 37 << 15;  // 1212416 = 296 tiles of 4096: one wave of 2 blocks per SM
+inline int sort_items(int64_t N) { return N >= kHugeTileKeys ? 32 : N >= kBigTileKeys ? 16 : 8; }
+// Dynamic shared memory of a sort pass: the staged tile (keys, values) and,
+// for 32 keys per thread, the ranks (registers would not hold them).
+inline size_t sort_pass_smem(int items) {
+  const size_t tile = static_cast<size_t>(kSortThreads) * items;
+  return tile * 8 + (items > 16 ? tile * 2 : 0);
+}
 constexpr int kMaxPasses = 4;
 constexpr int kGroupBits = 5;                         // 32 tiles per group, 32 groups per supergroup
 constexpr uint32_t kReady = 0x80000000u;              // look-back word: READY | count (count < 2^31)
-
-// Lanes of the warp holding the same BITS-bit value as this lane (valid
-// lanes only): one ballot per bit, each lane keeping the lanes that agree
-// with it on that bit.
-template <int BITS>
-__device__ __forceinline__ unsigned peers_of(bool valid, uint32_t value) {
-  unsigned peers = __ballot_sync(kFull, valid);
-#pragma unroll
-  for (int bit = 0; bit < BITS; ++bit) {
-    const bool set = (value >> bit) & 1u;
-    const unsigned m = __ballot_sync(kFull, set);
-    peers &= set ? m : ~m;
-  }
-  return valid ? peers : 0u;
-}
 
 // Block-wide exclusive sum (every thread passes one value); *total gets the sum.
 __device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t x, uint32_t* warp_tot, uint32_t* total) {
@@ -284,8 +278,10 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   constexpr int kSortTile = kSortThreads * ITEMS;   // positions per tile
   constexpr int kWarpSpan = kSortTile / kSortWarps;  // positions per warp within a tile
   __shared__ uint32_t wh[kSortWarps][kRadix];
-  __shared__ uint32_t stage_k[kSortTile];
-  __shared__ uint32_t stage_v[kSortTile];
+  extern __shared__ __align__(16) uint32_t sort_dyn[];
+  uint32_t* stage_k = sort_dyn;               // [kSortTile]
+  uint32_t* stage_v = sort_dyn + kSortTile;   // [kSortTile]
+  uint16_t* rank_s = reinterpret_cast<uint16_t*>(sort_dyn + 2 * kSortTile);  // [kSortTile], ITEMS > 16 only
   __shared__ uint32_t base_s[kRadix];
   __shared__ uint32_t start_s[kRadix];
   __shared__ uint32_t warp_tot[kSortWarps];
@@ -343,19 +339,36 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   uint32_t tile_n;
   const uint32_t local_start = block_exclusive_sum(count, warp_tot, &tile_n);
   if (tid < kRadix) start_s[tid] = local_start;
-  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) (&wh[0][0])[k] = 0;
+  uint32_t* match = stage_k + warp * kRadix;  // free until the tile is staged: one lane mask per digit and warp
+  for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads) {
+    (&wh[0][0])[k] = 0;
+    stage_k[k] = 0;
+  }
   __syncthreads();
-  // rank among the same digit within the warp's positions, in order
-  uint16_t rank[ITEMS];
+  // rank among the same digit within the warp's positions, in order: the
+  // lanes holding one digit find each other by OR-ing their bit into the
+  // digit's mask (three shared-memory operations instead of eight ballots:
+  // the ranking was ALU-bound)
+  constexpr bool kRankInSmem = ITEMS > 16;
+  uint16_t rank[kRankInSmem ? 1 : ITEMS];
 #pragma unroll
   for (int r = 0; r < ITEMS; ++r) {
     const bool valid = i0 + r * 32 + lane < N;
     const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-    const unsigned peers = peers_of<8>(valid, digit);
-    const unsigned lower = __popc(peers & lanemask_lt());
-    rank[r] = valid ? static_cast<uint16_t>(wh[warp][digit] + lower) : 0;  // < 512 keys per warp
+    if (valid) atomicOr(match + digit, 1u << lane);
     __syncwarp();
-    if (valid && lower == 0) wh[warp][digit] += __popc(peers);
+    const unsigned peers = valid ? match[digit] : 0u;
+    const unsigned lower = __popc(peers & lanemask_lt());
+    const uint16_t rk = valid ? static_cast<uint16_t>(wh[warp][digit] + lower) : 0;  // < kWarpSpan
+    if constexpr (kRankInSmem)
+      rank_s[warp * kWarpSpan + r * 32 + lane] = rk;
+    else
+      rank[r] = rk;
+    __syncwarp();
+    if (valid && lower == 0) {
+      wh[warp][digit] += __popc(peers);
+      match[digit] = 0;
+    }
     __syncwarp();
   }
   __syncthreads();
@@ -374,7 +387,12 @@ __global__ void __launch_bounds__(kSortThreads, ITEMS > 8 ? 2 : 3) sort_pass_ker
   for (int r = 0; r < ITEMS; ++r) {
     if (i0 + r * 32 + lane < N) {
       const uint32_t digit = (key[r] >> shift) & (kRadix - 1);
-      const uint32_t pos = start_s[digit] + wh[warp][digit] + rank[r];
+      uint32_t rk;
+      if constexpr (kRankInSmem)
+        rk = rank_s[warp * kWarpSpan + r * 32 + lane];
+      else
+        rk = rank[r];
+      const uint32_t pos = start_s[digit] + wh[warp][digit] + rk;
       stage_k[pos] = key[r];
       stage_v[pos] = val[r];
     }
@@ -488,11 +506,16 @@ inline ple_status_t launch_sort(const int64_t* rows, int64_t N, int64_t num_rows
   e = launch_after(key_hist_kernel, dim3(static_cast<unsigned>(hist_blocks)), dim3(kSortThreads), 0, s, rows,
                    num_rows, sa, run_done, nwin);
   if (e != cudaSuccess) return cuda_fail(e);
+  const size_t smem = sort_pass_smem(L.items);
+  if (L.items == 32) {
+    e = cudaFuncSetAttribute(sort_pass_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   for (int p = 0; p < sa.passes; ++p) {
-    e = L.items > 8 ? launch_after(sort_pass_kernel<16>, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s,
-                                   sa, p)
-                    : launch_after(sort_pass_kernel<8>, dim3(static_cast<unsigned>(L.tiles)), dim3(kSortThreads), 0, s,
-                                   sa, p);
+    const dim3 grid(static_cast<unsigned>(L.tiles));
+    e = L.items == 32   ? launch_after(sort_pass_kernel<32>, grid, dim3(kSortThreads), smem, s, sa, p)
+        : L.items == 16 ? launch_after(sort_pass_kernel<16>, grid, dim3(kSortThreads), smem, s, sa, p)
+                        : launch_after(sort_pass_kernel<8>, grid, dim3(kSortThreads), smem, s, sa, p);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   *sorted_keys = sa.keys[sa.passes & 1];

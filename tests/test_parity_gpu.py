@@ -177,10 +177,11 @@ def test_gradient_many_tiles(cuda_device, D, gdt):
     check_backward(w, cuda_device, rows)
 
 
-@pytest.mark.parametrize("N", [3 * 2**17 - 1, 3 * 2**17 + 777])
+@pytest.mark.parametrize("N", [3 * 2**17 - 1, 3 * 2**17 + 777, 37 * 2**15 - 1, 37 * 2**15 + 4097])
 def test_gradient_both_sort_tile_sizes(cuda_device, N):
-    """Just below and above the key count at which the sort passes switch
-    from 2048-key to 4096-key tiles (ragged last tile on both sides)."""
+    """Just below and above the key counts at which the sort passes switch
+    from 2048-key to 4096-key tiles and from 4096-key to 8192-key tiles
+    (ragged last tile on both sides)."""
     rng = np.random.default_rng(N)
     R = 1_000_003
     rows = synth.zipf_ids(N, 1.2, R, rng)
