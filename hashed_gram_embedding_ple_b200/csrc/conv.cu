@@ -174,6 +174,12 @@ struct ChainTaps {
       ahead = static_cast<int>(min(rem, static_cast<int64_t>(K - 1)));
     }
   }
+  // n steps inside the segment, each with all K - 1 taps behind and ahead
+  __device__ __forceinline__ void skip(int n) {
+    back = K - 1;
+    rem -= n;
+    ahead = rem < K - 1 ? static_cast<int>(rem) : K - 1;
+  }
 };
 
 // Block (0, 0) checks cu_seqlens once per launch: cu[0] == 0, cu[S] == T,
@@ -230,26 +236,48 @@ conv_forward_kernel(const unsigned char* __restrict__ x, int64_t T, int64_t nvec
         const int64_t t = tb + m * d;
         cur[m] = t < t1 ? ld_vec(xc + t * row) : make_uint4(0, 0, 0, 0);
       }
+      // interior iteration: every token of it, with all K taps, inside the
+      // chunk and one segment; then no per-token segment test (same sums)
+      sg.advance(tb);
+      const bool interior = tb + (U - 1) * d < t1 && tb - (K - 1) * d >= sg.lo && tb + (U - 1) * d < sg.hi;
+      if (interior) {
 #pragma unroll
-      for (int m = 0; m < U; ++m) {
-        const int64_t t = tb + m * d;
-        if (t < t1) {
-          sg.advance(t);
-          const int64_t seg_lo = sg.first(t);
+        for (int m = 0; m < U; ++m) {
           float acc[V];
 #pragma unroll
           for (int v = 0; v < V; ++v) acc[v] = b[v];
 #pragma unroll
           for (int k = 0; k < K; ++k) {
-            const int j = K - 1 - k;  // chain steps back
-            if (t - j * d >= seg_lo) {  // before the segment: zero history
-              float xv[V];
-              unpack<BF16>(m - j >= 0 ? cur[m - j] : prev[K + m - j], xv);
+            const int j = K - 1 - k;
+            float xv[V];
+            unpack<BF16>(m - j >= 0 ? cur[m - j] : prev[K + m - j], xv);
 #pragma unroll
-              for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], xv[v], acc[v]);
-            }
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], xv[v], acc[v]);
           }
-          st_cs(yc + t * row, pack<BF16>(acc));
+          st_cs(yc + (tb + m * d) * row, pack<BF16>(acc));
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < U; ++m) {
+          const int64_t t = tb + m * d;
+          if (t < t1) {
+            sg.advance(t);
+            const int64_t seg_lo = sg.first(t);
+            float acc[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = b[v];
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+              const int j = K - 1 - k;  // chain steps back
+              if (t - j * d >= seg_lo) {  // before the segment: zero history
+                float xv[V];
+                unpack<BF16>(m - j >= 0 ? cur[m - j] : prev[K + m - j], xv);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(wr[v][k], xv[v], acc[v]);
+              }
+            }
+            st_cs(yc + t * row, pack<BF16>(acc));
+          }
         }
       }
 #pragma unroll
@@ -470,11 +498,14 @@ conv_backward_kernel(const unsigned char* __restrict__ dy, const unsigned char* 
         xq[m] = t < t1 ? ld_quad<BF16>(xc + t * row) : zero_quad<BF16>();
         gq[m] = tg < T && t < t1 ? ld_quad<BF16>(gc + tg * row) : zero_quad<BF16>();
       }
+      // interior iteration: its K tokens inside the chunk, and every one with
+      // all K taps behind and ahead inside the segment of the previous chain
+      // step; then no per-token segment bookkeeping or tap tests (same sums)
+      const bool interior = tb + (U - 1) * d < t1 && tb - static_cast<int64_t>(L) * d >= ct.lo &&
+                            tb - d >= ct.lo && tb + static_cast<int64_t>(U - 1 + L) * d < ct.hi;
+      if (interior) {
 #pragma unroll
-      for (int m = 0; m < U; ++m) {
-        const int64_t t = tb + m * d;
-        if (t < t1) {
-          ct.step(sg, t, d);
+        for (int m = 0; m < U; ++m) {
           float g[4];
           unpack4<BF16>(m < L ? ga[m] : gn[m - L], g);
 #pragma unroll
@@ -482,26 +513,59 @@ conv_backward_kernel(const unsigned char* __restrict__ dy, const unsigned char* 
 #pragma unroll
           for (int k = 0; k < K; ++k) {
             const int j = K - 1 - k;
-            if (j <= ct.back) {  // output t read x[t - j d] through tap k
-              float xv[4];
-              unpack4<BF16>(m - j >= 0 ? xn[m - j] : xp[L + m - j], xv);
+            float xv[4];
+            unpack4<BF16>(m - j >= 0 ? xn[m - j] : xp[L + m - j], xv);
 #pragma unroll
-              for (int v = 0; v < 4; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
-            }
+            for (int v = 0; v < 4; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
           }
           if (dx != nullptr) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k = 0; k < K; ++k) {
               const int j = K - 1 - k;
-              if (j <= ct.ahead) {  // x[t] fed output t + j d through tap k
-                float gv[4];
-                unpack4<BF16>(m + j < L ? ga[m + j] : gn[m + j - L], gv);
+              float gv[4];
+              unpack4<BF16>(m + j < L ? ga[m + j] : gn[m + j - L], gv);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+              for (int v = 0; v < 4; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+            }
+            st_quad<BF16>(dxc + (tb + m * d) * row, acc);
+          }
+        }
+        ct.skip(U);
+      } else {
+#pragma unroll
+        for (int m = 0; m < U; ++m) {
+          const int64_t t = tb + m * d;
+          if (t < t1) {
+            ct.step(sg, t, d);
+            float g[4];
+            unpack4<BF16>(m < L ? ga[m] : gn[m - L], g);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) gb[v] += g[v];
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+              const int j = K - 1 - k;
+              if (j <= ct.back) {  // output t read x[t - j d] through tap k
+                float xv[4];
+                unpack4<BF16>(m - j >= 0 ? xn[m - j] : xp[L + m - j], xv);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) gw[v][k] = fmaf(g[v], xv[v], gw[v][k]);
               }
             }
-            st_quad<BF16>(dxc + t * row, acc);
+            if (dx != nullptr) {
+              float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int k = 0; k < K; ++k) {
+                const int j = K - 1 - k;
+                if (j <= ct.ahead) {  // x[t] fed output t + j d through tap k
+                  float gv[4];
+                  unpack4<BF16>(m + j < L ? ga[m + j] : gn[m + j - L], gv);
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) acc[v] = fmaf(wr[v][k], gv[v], acc[v]);
+                }
+              }
+              st_quad<BF16>(dxc + t * row, acc);
+            }
           }
         }
       }
