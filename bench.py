@@ -384,12 +384,14 @@ def main():
     ap.add_argument("--conv-channels", type=int, default=8192, help="channels of the --conv workload")
     ap.add_argument("--host-table", action="store_true",
                     help="keep the table in pinned host memory: time ple_prefetch, the cached lookup and gradient, "
-                         "and the two-stream pipeline")
+                         "and the two-stream pipeline (single_layer_bf16 unless --workload names another)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.workload == "headline" and (args.fwd_only or args.slice or args.host_table):
-        raise SystemExit("--fwd-only, --slice and --host-table need a single --workload")
+    if args.host_table and args.workload == "headline":
+        args.workload = "single_layer_bf16"  # the host-table mode's own default (a 2 GB table, pinned)
+    if args.workload == "headline" and (args.fwd_only or args.slice):
+        raise SystemExit("--fwd-only and --slice need a single --workload")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

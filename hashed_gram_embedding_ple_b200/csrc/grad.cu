@@ -10,7 +10,8 @@
 //   added once into table_grad[r].
 //
 // Pipeline (all in the caller's workspace, no allocation):
-//   0. clear_kernel: zeroes the digit totals and the tile tickets;
+//   0. clear_kernel: zeroes the digit totals, the tile tickets and the
+//      call's abort word;
 //   1. key_hist_kernel: 32-bit keys from the int64 rows (bad rows -> key R)
 //      and the digit counts of every radix pass;
 //   2. sort_pass_kernel, once per 8-bit digit: LSD radix sort, stable,
@@ -21,8 +22,12 @@
 //      whole single-chunk run into table_grad, or stores the chunk sum of a
 //      longer run in a slot; the writer that completes a long run (per-run
 //      counter) folds that run's chunk sums in order and adds the result.
-// The final add is a vector fp32 reduction (red.global.add) issued by the one
-// warp that owns the row, so it is the single add table_grad + S_r.
+//      If a wait of the sort gave up (the call's abort word is set), the
+//      fold writes nothing.
+// The final add is made once per row by the lanes that own it: a vector fp32
+// reduction (red.global.add) when that gives the IEEE sum, else a plain
+// IEEE add (subnormals: see the comment above any_tiny), so it is the single
+// add table_grad + S_r.
 #include <algorithm>
 #include <atomic>
 

@@ -154,11 +154,14 @@ unsigned int* status_word(const ple_plan_t* plan, cudaStream_t stream, cudaError
   unsigned int* w = words + plan->status_slot;
   // the slot may hold bits of a destroyed plan that had it before: cleared
   // (in stream order, ahead of this call's kernels) on the plan's first call
-  // in each device context
-  if (plan->cleared_ctx[dev].load(std::memory_order_acquire) != ctx) {
+  // in each device context, by the one thread that claims that first call
+  unsigned long long seen = plan->cleared_ctx[dev].load(std::memory_order_acquire);
+  if (seen != ctx && plan->cleared_ctx[dev].compare_exchange_strong(seen, ctx, std::memory_order_acq_rel)) {
     *err = cudaMemsetAsync(w, 0, sizeof(unsigned int), stream);
-    if (*err != cudaSuccess) return nullptr;
-    plan->cleared_ctx[dev].store(ctx, std::memory_order_release);
+    if (*err != cudaSuccess) {
+      plan->cleared_ctx[dev].store(~0ull, std::memory_order_release);
+      return nullptr;
+    }
   }
   return w;
 }

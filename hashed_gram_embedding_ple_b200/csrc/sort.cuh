@@ -221,17 +221,18 @@ struct SortArgs {
   WaitCtl wc;              // bounded waits; wc.abort is zeroed before the sort with hist and tickets
 };
 
-// Keys from the int64 rows (a row outside [0, num_rows) becomes the key
-// num_rows, sorted last and skipped by the fold) and the digit counts of
-// every pass.  Also clears the look-back words of every pass and the fold's
-// run counters.
-// Clears the digit totals and tile tickets before key_hist_kernel adds to them.
+// Clears the digit totals, the tile tickets and the call's abort word
+// before key_hist_kernel adds to them.
 __global__ void clear_kernel(uint32_t* words, int n) {
   wait_for_prior_grid();  // (launched early, behind the caller's previous kernel)
   for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0;
   allow_next_grid();
 }
 
+// Keys from the int64 rows (a row outside [0, num_rows) becomes the key
+// num_rows, sorted last and skipped by the fold) and the digit counts of
+// every pass.  Also clears the look-back words of every pass and the fold's
+// run counters.
 __global__ void __launch_bounds__(kSortThreads)
 key_hist_kernel(const int64_t* __restrict__ rows, int64_t num_rows, const SortArgs a, unsigned int* run_done,
                 int64_t nwin) {

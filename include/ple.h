@@ -324,8 +324,13 @@ ple_status_t ple_conv_backward(const void* dy, const void* x, ple_dtype_t dtype,
  * flags alone.  plan == NULL takes every word of the device at once: the
  * flags of all plans and of the calls that take no plan (the short
  * convolution).  Synchronises `stream` (the only call that does); not for
- * use inside a stream capture.  Device addresses are looked up again after
- * the current context changes (cudaDeviceReset). */
+ * use inside a stream capture.  A plan's word is cleared, in stream order,
+ * by the plan's first call on each device (a destroyed plan's unread flags
+ * are not inherited); a plan about to be used from several host threads on
+ * several streams should make one call on each device first, so that this
+ * clear cannot land after another stream's kernel has raised a flag.
+ * Device addresses are looked up again after the current context changes
+ * (cudaDeviceReset). */
 ple_status_t ple_status(const ple_plan_t* plan, void* stream);
 
 /* Text for a status code (static storage). */
