@@ -294,8 +294,9 @@ size_t ple_conv_backward_workspace_bytes(int64_t num_tokens, int64_t channels, i
  *              the segment), dbias[c] += sum_t dy[t, c] (fp32, accumulated
  *              into; NULL to skip).
  * The sums over tokens have a fixed order, so results are bit-identical run
- * to run: the tokens are cut into consecutive chunks (at least 256 tokens,
- * at most 1024 chunks); each chunk's sum starts from +0 and adds its tokens
+ * to run: the tokens are cut into consecutive chunks (256 tokens, or 512
+ * when ceil(num_tokens / 512) * ceil(channels / 512) >= 592; more when that
+ * would exceed 1024 chunks); each chunk's sum starts from +0 and adds its tokens
  * residue class by residue class modulo the dilation (the class of the
  * chunk's first token first), each class in ascending token order (fused
  * multiply-add for dweight); the chunk sums are added in chunk order

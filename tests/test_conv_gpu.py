@@ -4,9 +4,9 @@ depthwise) through the C ABI against the oracle.
 Tolerances follow from the arithmetic: an output is an fp32 sum of at most
 K + 1 terms (at most K + 1 roundings of at most 2^-24 of the magnitude sum
 mag = |b| + sum |w x|), then rounded to the output type (bf16: half an ulp,
-at most 2^-8 of the value); dw and db are fp32 sums over chunks of at most
-256 tokens added in chunk order (at most 1024 chunks), well inside 2^-14 of
-their magnitude sums.
+at most 2^-8 of the value); dw and db are fp32 sums over chunks of 256 or
+512 tokens added in chunk order (at most 1024 chunks): at most (512 + 1024)
+roundings of 2^-24 of their magnitude sums, inside 2^-14 of them.
 """
 import numpy as np
 import pytest
