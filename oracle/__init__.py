@@ -44,8 +44,11 @@ def build(force: bool = False, sanitize: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(LIB_PATH)
+        # PLE_ORACLE_SANITIZED=1 loads the ASan/UBSan build (the process must
+        # then preload the sanitizer runtimes; see tests/test_oracle_pins.py)
+        sanitized = os.environ.get("PLE_ORACLE_SANITIZED") == "1"
+        path = build(sanitize=sanitized)
+        lib = ctypes.CDLL(path)
         lib.oracle_ple_rows.argtypes = [_i64p, ctypes.c_int64, _i32p, ctypes.c_int32, ctypes.c_int32,
                                         ctypes.c_int32, ctypes.c_int64, _i64p, _i64p, _i64p, _i64p]
         lib.oracle_ple_rows.restype = ctypes.c_int

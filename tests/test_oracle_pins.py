@@ -15,6 +15,9 @@
   element, one final add) produces.
 """
 import itertools
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -22,7 +25,7 @@ import torch
 
 import oracle
 import synth
-from conftest import read_golden_blocks
+from conftest import ROOT, read_golden_blocks
 
 pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
 
@@ -535,3 +538,77 @@ def test_conv_backward_matches_autograd_and_adjoint():
         dxi, dwi, _ = oracle.conv_backward(gi, xi, cu, wi, d)
         assert float((oracle.conv_forward(xi, cu, wi, d) * gi).sum()) == float((xi * dxi).sum())
         assert float((oracle.conv_forward(xi, cu, wi, d) * gi).sum()) == float((wi * dwi).sum())
+
+
+# ---------------------------------------------------------------------------
+# the oracle under AddressSanitizer / UndefinedBehaviorSanitizer
+# ---------------------------------------------------------------------------
+
+_SANITIZED_RUN = r"""
+import hashlib, sys
+import numpy as np
+sys.path.insert(0, sys.argv[1])
+import oracle, synth
+h = hashlib.sha256()
+rng = np.random.default_rng(3)
+for n, G in ((2, 1), (3, 2), (4, 3)):
+    lens = [0, 1, 7, 300, 0, 55]
+    tok = rng.integers(0, 20, sum(lens))
+    cu = synth.cu_seqlens_from_lengths(lens)
+    mults = synth.signed_mults(n, rng)
+    primes = synth.consecutive_primes(97, (n - 1) * G)
+    offs = synth.exclusive_prefix(primes)
+    rows = oracle.rows(tok, cu, n, G, 0, mults, primes, offs)
+    rows_mt = oracle.rows(tok, cu, n, G, 0, mults, primes, offs, threads=3)
+    table = rng.standard_normal((int(sum(primes)), 8)).astype(np.float32)
+    out = oracle.gather(rows, table)
+    codes = rng.integers(0, 256, (int(sum(primes)), 16)).astype(np.uint8)
+    wide = oracle.gather_e4m3(rows, codes)
+    g = rng.standard_normal((rows.size, 8)).astype(np.float32)
+    uniq, sums = oracle.grad_sums(rows, g)
+    _, sums_mt = oracle.grad_sums(rows, g, threads=3)
+    tg = oracle.grad_apply(rows, g, np.zeros_like(table))
+    x = rng.standard_normal((len(tok), 5))
+    dy = rng.standard_normal((len(tok), 5))
+    w = rng.standard_normal((5, 4))
+    y = oracle.conv_forward(x, cu, w, n, rng.standard_normal(5))
+    dx, dw, db = oracle.conv_backward(dy, x, cu, w, n)
+    for a in (rows, rows_mt, out, wide, uniq, sums, sums_mt, tg, y, dx, dw, db):
+        h.update(np.ascontiguousarray(a).tobytes())
+print(h.hexdigest())
+"""
+
+
+def _libs_exist():
+    import shutil
+
+    if shutil.which("gcc") is None:
+        return None
+    out = []
+    for lib in ("libasan.so", "libubsan.so"):
+        p = subprocess.run(["gcc", f"-print-file-name={lib}"], capture_output=True, text=True).stdout.strip()
+        if not os.path.isabs(p) or not os.path.exists(p):
+            return None
+        out.append(p)
+    return out
+
+
+def test_oracle_clean_under_asan_and_ubsan():
+    """The oracle built with -fsanitize=address,undefined runs rows, gathers
+    (bf16 / fp32 / E4M3), gradient sums (one and several threads) and the
+    conv on ragged inputs (empty and one-token segments) without a report,
+    and gives the same bytes as the normal build."""
+    libs = _libs_exist()
+    if libs is None:
+        pytest.skip("gcc sanitizer runtimes not found")
+    oracle.build(sanitize=True)
+    env = dict(os.environ, PLE_ORACLE_SANITIZED="1", LD_PRELOAD=":".join(libs),
+               ASAN_OPTIONS="detect_leaks=0:verify_asan_link_order=0:halt_on_error=1",
+               UBSAN_OPTIONS="halt_on_error=1:print_stacktrace=1")
+    r = subprocess.run([sys.executable, "-c", _SANITIZED_RUN, ROOT], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-4000:]
+    assert "runtime error" not in r.stderr and "AddressSanitizer" not in r.stderr, r.stderr[-4000:]
+    plain = subprocess.run([sys.executable, "-c", _SANITIZED_RUN, ROOT], capture_output=True, text=True, timeout=600)
+    assert plain.returncode == 0, plain.stderr[-2000:]
+    assert r.stdout.strip() == plain.stdout.strip()

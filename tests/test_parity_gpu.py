@@ -341,3 +341,93 @@ def test_prepare_then_apply_equals_scatter(cuda_device):
     assert ple.ple_status() == ple.PLE_OK
     assert out.shape == (w.num_tokens, w.num_heads, w.head_dim)
     assert torch.equal(tg.view(torch.int32), ref.view(torch.int32))
+
+
+def _poison(ws, fill, seed=0):
+    if fill == "random":
+        g = torch.Generator(device=ws.device).manual_seed(seed)
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device=ws.device, generator=g))
+    else:
+        ws.fill_(fill)
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, "random"])
+@pytest.mark.parametrize("N", [3 * 4096 + 1234, 3 * 2**17 + 5, 37 * 2**15 + 999])
+def test_gradient_workspace_contents_do_not_matter(cuda_device, fill, N):
+    """The caller's workspace may hold anything (a reused buffer, bytes left
+    by another call): every word the gradient needs cleared (digit totals,
+    tile tickets, the abort word, look-back rows, run counters) is cleared by
+    the call itself.  All three sort tile sizes; ple_grad_scatter and the
+    prepare / apply halves, against the oracle."""
+    dev = cuda_device
+    rng = np.random.default_rng(N)
+    R = 1_000_003
+    rows = synth.zipf_ids(N, 1.2, R, rng)
+    w = custom_workload("poison", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [R], 16, synth.DTYPE_F32,
+                        synth.DTYPE_BF16, seed=N % 97)
+    plan = ple.Plan.from_workload(w)
+    g_host = host_grad(w, N)
+    g = values_to_torch(g_host, w.grad_dtype).to(dev)
+    rows_d = dev_i64(rows, dev)
+    ref = oracle.grad_apply(rows, g_host, np.zeros((R, 16), np.float32))
+    ws = ple.alloc_workspace(plan, N, dev)
+    _poison(ws, fill, seed=1)
+    tg = torch.zeros(R, 16, device=dev)
+    ple.ple_grad_scatter(plan, rows_d, g, tg, workspace=ws)
+    assert ple.ple_status(dev, plan=plan) == ple.PLE_OK
+    np.testing.assert_array_equal(tg.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    _poison(ws, fill, seed=2)
+    tg.zero_()
+    ple.ple_grad_prepare(plan, rows_d, ws)
+    ple.ple_grad_apply(plan, N, g, tg, ws)
+    assert ple.ple_status(dev, plan=plan) == ple.PLE_OK
+    np.testing.assert_array_equal(tg.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("fill", [0xFF, "random"])
+def test_prefetch_and_conv_workspace_contents_do_not_matter(cuda_device, fill):
+    """ple_prefetch and ple_conv_backward give the same bits with a poisoned
+    workspace as with a zeroed one."""
+    dev = cuda_device
+    rng = np.random.default_rng(77)
+    lens = [300, 0, 4000, 1, 2500]
+    tok = rng.integers(0, 200, sum(lens))
+    w = custom_workload("pf_poison", tok, synth.cu_seqlens_from_lengths(lens), 3, 4, 0, synth.signed_mults(3, rng),
+                        synth.consecutive_primes(5003, 8), 32, synth.DTYPE_BF16, synth.DTYPE_BF16)
+    plan = ple.Plan.from_workload(w)
+    host_table, _ = small_table(w, dev)
+    pinned = values_to_torch(host_table, w.table_dtype).pin_memory()
+    tok_d, cu_d = dev_i64(w.tokens, dev), dev_i32(w.cu_seqlens, dev)
+    outs = []
+    for poison in (False, True):
+        buf = ple.Prefetched(plan, w.num_tokens, dev)
+        if poison:
+            _poison(buf.workspace, fill, seed=3)
+        else:
+            buf.workspace.zero_()
+        ple.ple_prefetch(plan, tok_d, cu_d, pinned, buf)
+        assert ple.ple_status(dev, plan=plan) == ple.PLE_OK
+        U = int(buf.num_unique.item())
+        outs.append((U, buf.slots.clone(), buf.uniq_rows[:U].clone(), buf.cache[:U].clone()))
+    assert outs[0][0] == outs[1][0]
+    for a, b in zip(outs[0][1:], outs[1][1:]):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    # conv backward: partial-sum workspace
+    T, C, K, d = sum(lens), 64, 4, 3
+    x = torch.from_numpy(rng.standard_normal((T, C)).astype(np.float32)).to(dev)
+    dy = torch.from_numpy(rng.standard_normal((T, C)).astype(np.float32)).to(dev)
+    wt = torch.from_numpy(rng.standard_normal((C, K)).astype(np.float32)).to(dev)
+    cu = dev_i32(synth.cu_seqlens_from_lengths(lens), dev)
+    res = []
+    for poison in (False, True):
+        ws = torch.empty(ple.conv_workspace_bytes(T, C, K), dtype=torch.uint8, device=dev)
+        if poison:
+            _poison(ws, fill, seed=4)
+        else:
+            ws.zero_()
+        dw, db = torch.zeros(C, K, device=dev), torch.zeros(C, device=dev)
+        dx, _, _ = ple.conv_backward(dy, x, cu, wt, d, dweight=dw, dbias=db, workspace=ws)
+        res.append((dx, dw, db))
+    assert ple.ple_status(dev) == ple.PLE_OK
+    for a, b in zip(*res):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
