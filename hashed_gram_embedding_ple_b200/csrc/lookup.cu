@@ -10,6 +10,8 @@
 // lanes.  UNROLL independent loads are in flight per thread before the
 // matching stores are issued.  An fp8 E4M3 table is widened to bf16 on the
 // way (8 bytes of codes in, 16 bytes of bf16 out per unit).
+#include <atomic>
+
 #include "common.cuh"
 
 namespace ple {
@@ -420,9 +422,19 @@ ple_status_t ple_hash(const ple_plan_t* plan, const int64_t* tokens, int64_t T, 
   if (status == nullptr) return cuda_fail(e);
   const int H = plan->hp.num_heads;
   const size_t smem = H * sizeof(HeadConst) + static_cast<size_t>(kHashWarps) * 32 * H * sizeof(int64_t);
-  if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(hash_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (smem > 48 * 1024) {  // once per device and context, for the largest size a plan can ask for
+    static std::atomic<unsigned long long> allowed[64];  // context id + 1, per device
+    int dev = 0;
+    e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
+    unsigned long long ctx = 0;
+    current_context_id(&ctx);
+    if (dev >= 64 || allowed[dev].load(std::memory_order_acquire) != ctx + 1) {
+      const size_t most = kMaxHeads * sizeof(HeadConst) + static_cast<size_t>(kHashWarps) * 32 * kMaxHeads * sizeof(int64_t);
+      e = cudaFuncSetAttribute(hash_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(most));
+      if (e != cudaSuccess) return cuda_fail(e);
+      if (dev < 64) allowed[dev].store(ctx + 1, std::memory_order_release);
+    }
   }
   const int64_t warps = (T + 31) / 32;
   const dim3 grid(static_cast<unsigned>((warps + kHashWarps - 1) / kHashWarps));

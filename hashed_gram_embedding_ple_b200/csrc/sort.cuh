@@ -508,9 +508,19 @@ inline ple_status_t launch_sort(const int64_t* rows, int64_t N, int64_t num_rows
                    num_rows, sa, run_done, nwin);
   if (e != cudaSuccess) return cuda_fail(e);
   const size_t smem = sort_pass_smem(L.items);
-  if (L.items == 32) {
-    e = cudaFuncSetAttribute(sort_pass_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (L.items == 32) {  // more than 48 KB of dynamic shared memory: allowed once per device and context
+    static std::atomic<unsigned long long> allowed[64];  // context id + 1, per device
+    int dev = 0;
+    e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
+    unsigned long long ctx = 0;
+    current_context_id(&ctx);
+    if (dev >= 64 || allowed[dev].load(std::memory_order_acquire) != ctx + 1) {
+      e = cudaFuncSetAttribute(sort_pass_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sort_pass_smem(32)));
+      if (e != cudaSuccess) return cuda_fail(e);
+      if (dev < 64) allowed[dev].store(ctx + 1, std::memory_order_release);
+    }
   }
   for (int p = 0; p < sa.passes; ++p) {
     const dim3 grid(static_cast<unsigned>(L.tiles));
