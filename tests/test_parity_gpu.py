@@ -92,6 +92,7 @@ def test_tiny_forward_backward(cuda_device):
     (5, 4, 64, synth.DTYPE_F32),
     (8, 1, 256, synth.DTYPE_BF16),   # largest order
     (3, 32, 32, synth.DTYPE_F32),    # 64 heads
+    (3, 32, 256, synth.DTYPE_F32),   # 64 heads of 1 KB rows: one token per warp, the generic fold at D = 256
 ])
 def test_ragged_multi_tile(cuda_device, n, G, D, dt):
     rng = np.random.default_rng(100 + n * 10 + G)
