@@ -341,9 +341,10 @@ class Part:
 
     def launches(self):
         """Kernels per step: the lookup; the backward's clear, key_hist, one
-        sort pass per 8-bit digit of the row ids, and the fold."""
+        sort pass per 8-bit digit of the row ids, the fold and the long-run
+        finish."""
         passes = max(1, (int(self.w.num_rows).bit_length() + 7) // 8)
-        return 1 + (3 + passes if self.do_bwd else 0)
+        return 1 + (4 + passes if self.do_bwd else 0)
 
     def fwd_bytes(self):
         w = self.w

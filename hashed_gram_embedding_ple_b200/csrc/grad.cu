@@ -21,7 +21,9 @@
 //      offset from its run's first position is a multiple of 32), adds a
 //      whole single-chunk run into table_grad, or stores the chunk sum of a
 //      longer run in a slot; the writer that completes a long run (per-run
-//      counter) folds that run's chunk sums in order and adds the result.
+//      counter) folds that run's chunk sums in order and adds the result;
+//   4. finish_long_runs_kernel: the same second level for the runs of more
+//      than kLongChunks chunks, which the fold lists instead (hot rows).
 //      If a wait of the sort gave up (the call's abort word is set), the
 //      fold writes nothing.
 // The final add is made once per row by the lanes that own it: a vector fp32
@@ -330,11 +332,33 @@ __device__ __forceinline__ bool window_setup(const uint32_t* __restrict__ K, con
 // order (second level) and makes the run's single final add.  Nobody waits.
 constexpr unsigned kDoneTarget = 1u << 30;
 
+// A run of more than kLongChunks chunks is not finished by the warp that
+// completes it (one warp would fold its chunk sums at one short batch per
+// memory round trip) but listed for finish_long_runs_kernel.
+// (Runs up to this length finish inside the fold at no visible cost: its other warps keep the memory
+// busy meanwhile; a 64-chunk threshold cost backward_stress, whose longest runs have 266 chunks, 10 us.)
+constexpr int kLongChunks = 512;
+
+struct LongRun {
+  int64_t s;     // first sorted position of the run
+  int32_t nc;    // its chunks
+  uint32_t key;  // its row
+};
+
 struct RunBook {
   int* len;               // [windows] run length, written by the last chunk's writer
   unsigned* done;         // [windows] completion counters, cleared before the fold
   const uint32_t* abort;  // the sort's abort word: non-zero, the fold writes nothing
+  LongRun* long_runs;     // [long_cap] runs left to finish_long_runs_kernel
+  unsigned* long_count;   // their count (cleared with the completion counters)
+  unsigned long_cap;
 };
+
+// Lists a completed run for finish_long_runs_kernel (by one lane).
+__device__ __forceinline__ void list_long_run(const RunBook& rb, int64_t s, int nc, uint32_t key) {
+  const unsigned at = atomicAdd(rb.long_count, 1u);
+  if (at < rb.long_cap) rb.long_runs[at] = LongRun{s, nc, key};  // (always: long_cap bounds the runs)
+}
 
 __device__ __forceinline__ int64_t chunk_slot(int64_t s, int m) {
   return m == 0 ? 2 * (s >> 5) + 1 : 2 * ((s + static_cast<int64_t>(m) * kChunk) >> 5);
@@ -598,9 +622,13 @@ fold_wide_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__ I,
         const unsigned gmask = L == 32 ? kFull : (((1u << L) - 1u) << (grp * L));
         int64_t s = 0;
         const int nc = chunk_stored(W, c, nxt, N, gmask, grp * L, rb, &s);
-        if (nc && sub == 0) {  // this chunk completed a long run: fold it once the window is done
-          const int at = atomicAdd(npend, 1);  // at most 2: a window holds chunks of at most 2 long runs
-          if (at < 2) pend[at] = PendingRun{s, nc, key};
+        if (nc && sub == 0) {  // this chunk completed a long run
+          if (nc > kLongChunks) {
+            list_long_run(rb, s, nc, key);
+          } else {  // fold it once the window is done
+            const int at = atomicAdd(npend, 1);  // at most 2: a window holds chunks of at most 2 long runs
+            if (at < 2) pend[at] = PendingRun{s, nc, key};
+          }
         }
       }
     }
@@ -666,7 +694,9 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
               store_slot<0>(csum, slot, D, acc);
               int64_t s = 0;
               const int nc = chunk_stored(W, c, nxt, N, kFull, 0, rb, &s);
-              if (nc) {  // second level by the whole warp, lanes owning columns l, l+32, ...
+              if (nc > kLongChunks) {
+                if (lane == 0) list_long_run(rb, s, nc, key);
+              } else if (nc) {  // second level by the whole warp, lanes owning columns l, l+32, ...
                 Cols<0> sum;
 #pragma unroll
                 for (int q = 0; q < Cols<0>::n; ++q) {
@@ -687,6 +717,67 @@ fold_generic_kernel(const uint32_t* __restrict__ K, const uint32_t* __restrict__
         }
       }
     }
+  }
+}
+
+// Second level of the listed long runs.  One block per (run, 32-column
+// slice): lane l of warp 0 owns column 32 g + l and adds the run's chunk sums
+// in order, left to right from the first (the order finish_run_staged uses),
+// then makes the run's single final add into table_grad.  All eight warps
+// stream the slice's chunk sums into a ring of kFinStages stages of
+// kFinStage slices in shared memory with asynchronous copies, kFinStages - 1
+// stages ahead (one warp alone keeps too few copies in flight), and the
+// slices of one run go to different SMs.
+constexpr int kFinThreads = 256;
+constexpr int kFinStage = 128;  // chunk sums per stage
+constexpr int kFinStages = 3;   // stages in the ring: 3 * 128 slices of 128 bytes = 48 KB
+constexpr size_t kFinSmem = static_cast<size_t>(kFinStages) * kFinStage * 32 * sizeof(float);
+
+__global__ void __launch_bounds__(kFinThreads)
+finish_long_runs_kernel(const LongRun* __restrict__ runs, const unsigned* __restrict__ count, unsigned cap,
+                        const float* __restrict__ csum, int D, float* __restrict__ table_grad,
+                        const uint32_t* abort) {
+  extern __shared__ __align__(16) float fin_ring[];  // [kFinStages][kFinStage][32]
+  wait_for_prior_grid();
+  if (ld_relaxed(abort) != 0) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int groups = (D + 31) / 32;
+  const int64_t items = static_cast<int64_t>(min(ld_relaxed(count), cap)) * groups;  // (count <= cap)
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const LongRun run = runs[item / groups];
+    const int c0 = 32 * static_cast<int>(item % groups);
+    const int cols = min(32, D - c0);  // a multiple of 4: grad rows are 16-byte multiples
+    const int vps = cols / 4;          // 16-byte vectors per slice
+    const int64_t nst = (run.nc + kFinStage - 1) / kFinStage;
+    auto load_stage = [&](int64_t k) {  // chunk sums k*S .. k*S+S-1 into stage k mod kFinStages
+      float* st = fin_ring + (k % kFinStages) * kFinStage * 32;
+      for (int idx = tid; idx < kFinStage * vps; idx += kFinThreads) {
+        const int i = idx / vps, v = idx - i * vps;
+        const int64_t m = k * kFinStage + i;
+        if (m < run.nc)
+          cp_async16(st + i * 32 + 4 * v, csum + chunk_slot(run.s, static_cast<int>(m)) * D + c0 + 4 * v);
+      }
+    };
+    for (int64_t k = 0; k < kFinStages - 1; ++k) {
+      if (k < nst) load_stage(k);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    float acc = 0.f;
+    for (int64_t k = 0; k < nst; ++k) {
+      if (k + kFinStages - 1 < nst) load_stage(k + kFinStages - 1);  // into the stage read at k - 1
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group %0;" ::"n"(kFinStages - 1) : "memory");  // this thread's part of stage k
+      __syncthreads();                                                            // everyone's part
+      if (warp == 0 && lane < cols) {
+        const float* st = fin_ring + (k % kFinStages) * kFinStage * 32;
+        const int cnt = static_cast<int>(min(static_cast<int64_t>(kFinStage), run.nc - k * kFinStage));
+        for (int i = 0; i < cnt; ++i) acc = (k == 0 && i == 0) ? st[i * 32 + lane] : acc + st[i * 32 + lane];
+      }
+      __syncthreads();  // the stage just read is refilled two iterations on
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (warp == 0 && lane < cols) red_add1<false>(table_grad + static_cast<int64_t>(run.key) * D + c0 + lane, acc);
+    __syncthreads();  // the next item's first stages overwrite the ring
   }
 }
 
@@ -715,8 +806,8 @@ atomic_kernel(const int64_t* __restrict__ rows, int64_t N, int64_t num_rows, con
 // ---------------------------------------------------------------------------
 struct Layout {
   SortLayout sort;
-  size_t csum, run_len, run_done, total_bytes;
-  int64_t nwin;
+  size_t csum, run_len, run_done, long_runs, total_bytes;
+  int64_t nwin, long_cap;
 };
 
 Layout layout_for(int64_t N, int D) {
@@ -731,7 +822,9 @@ Layout layout_for(int64_t N, int D) {
   };
   L.csum = take(sizeof(float) * 2 * static_cast<size_t>(L.nwin) * D);
   L.run_len = take(sizeof(int) * L.nwin);
-  L.run_done = take(sizeof(unsigned int) * L.nwin);
+  L.run_done = take(sizeof(unsigned int) * (L.nwin + 1));  // + the long-run count
+  L.long_cap = L.nwin / (kLongChunks + 1) + 1;  // a long run spans more than kLongChunks windows
+  L.long_runs = take(sizeof(LongRun) * static_cast<size_t>(L.long_cap));
   L.total_bytes = off;
   return L;
 }
@@ -808,10 +901,13 @@ ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, i
   rb.len = reinterpret_cast<int*>(ws + L.run_len);
   rb.done = reinterpret_cast<unsigned int*>(ws + L.run_done);
   rb.abort = sort_abort_word(L.sort, ws);
+  rb.long_count = rb.done + L.nwin;
+  rb.long_runs = reinterpret_cast<LongRun*>(ws + L.long_runs);
+  rb.long_cap = static_cast<unsigned>(L.long_cap);
   const uint32_t* Ks = nullptr;
   const uint32_t* Is = nullptr;
   if (phases & kPrepare) {
-    ple_status_t st = launch_sort(rows, N, num_rows, ws, L.sort, rb.done, L.nwin, status, s, &Ks, &Is);
+    ple_status_t st = launch_sort(rows, N, num_rows, ws, L.sort, rb.done, L.nwin + 1, status, s, &Ks, &Is);
     if (st != PLE_OK) return st;
     if (!(phases & kApply)) return check_launch();
   } else {
@@ -838,6 +934,13 @@ ple_status_t grad_scatter_bounded(const ple_plan_t* plan, const int64_t* rows, i
              : fold(fold_generic_kernel<false>, fold_grid, kFoldThreads, 0);
   }
 #undef PLE_WIDE
+  if (e != cudaSuccess) return cuda_fail(e);
+  // the long runs the fold listed (none in most calls: the blocks read the count and return)
+  const int64_t items = L.long_cap * ((D + 31) / 32);
+  const unsigned fin_blocks = static_cast<unsigned>(std::min<int64_t>(items, sm_count()));
+  e = launch_after(finish_long_runs_kernel, dim3(fin_blocks), dim3(kFinThreads), kFinSmem, s,
+                   static_cast<const LongRun*>(rb.long_runs), static_cast<const unsigned*>(rb.long_count),
+                   rb.long_cap, static_cast<const float*>(csum), D, table_grad, rb.abort);
   if (e != cudaSuccess) return cuda_fail(e);
   return check_launch();
 }

@@ -166,6 +166,20 @@ def test_gradient_chunk_boundaries(cuda_device):
     check_backward(w, cuda_device, rows, prefill=prefill)
 
 
+@pytest.mark.parametrize("D,gdt,N", [(128, synth.DTYPE_BF16, 300_001), (40, synth.DTYPE_F32, 300_001),
+                                     (64, synth.DTYPE_BF16, 512 * 32 + 50), (64, synth.DTYPE_BF16, 512 * 32 + 51)])
+def test_gradient_every_hit_on_one_row(cuda_device, D, gdt, N):
+    """The degenerate input of identical tokens: (nearly) every hit of the
+    call lands on one row, one run of up to 300,001 hits (9,376 chunk sums
+    folded in order by finish_long_runs_kernel), plus 50 hits on other rows;
+    the run of exactly 512 chunks stays inside the fold, 513 chunks do not."""
+    rng = np.random.default_rng(D + N)
+    rows = np.full(N, 7, np.int64)
+    rows[rng.choice(N, 50, replace=False)] = rng.integers(8, 40, 50)  # the hot row keeps exactly N - 50 hits
+    w = custom_workload("one_row", np.zeros(1, np.int64), [0, 1], 2, 1, 0, [1, 1], [41], D, synth.DTYPE_F32, gdt)
+    check_backward(w, cuda_device, rows)
+
+
 @pytest.mark.parametrize("D,gdt", [(32, synth.DTYPE_F32), (64, synth.DTYPE_BF16), (128, synth.DTYPE_BF16),
                                    (256, synth.DTYPE_F32), (40, synth.DTYPE_BF16), (200, synth.DTYPE_F32)])
 def test_gradient_many_tiles(cuda_device, D, gdt):
