@@ -161,7 +161,7 @@ __device__ __forceinline__ void copy_hits(const unsigned char* __restrict__ tabl
         const int hit = VL >= 0 ? (q >> VL) : q / V;
         const int col = q - hit * V;
         const int64_t off = rowoff[hit];
-        v[u] = off >= 0 ? ld_nc_na(table + off + col * 16) : make_uint4(0, 0, 0, 0);
+        v[u] = off >= 0 ? ld_nc(table + off + col * 16) : make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
@@ -237,7 +237,7 @@ __device__ __forceinline__ void widen_hits(const unsigned char* __restrict__ tab
         const int hit = VL8 >= 0 ? (q >> VL8) : q / V;
         const int col = q - hit * V;
         const int64_t off = rowoff[hit];
-        v[u] = off >= 0 ? ld_nc_na8(table + off + col * 8) : make_uint2(0, 0);
+        v[u] = off >= 0 ? ld_nc8(table + off + col * 8) : make_uint2(0, 0);
       }
     }
 #pragma unroll
