@@ -146,6 +146,41 @@ def traffic_from_profiles(key: str, source_files):
     return None
 
 
+def backward_split(p, flush_l2, stream, peak: float, reps: int = 10) -> dict:
+    """The backward of part p as its two halves, ple_grad_prepare (clear, key
+    histogram, sort passes) and ple_grad_apply (fold, long-run finish), timed
+    apart with CUDA events after the timed steps (L2 flushed before each
+    prepare).  The apply moves all of the backward's algorithmic bytes (the
+    sorted keys and hit ids in place of the row ids), so its GB/s is the
+    fold's own roofline figure; the prepare is the sort's overhead."""
+    import torch
+
+    N = p.T_out * p.w.num_heads
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for r in range(reps + 2):  # two untimed
+        flush_l2()
+        e = ev[r - 2] if r >= 2 else None
+        if e is not None:
+            e[0].record(stream)
+        p.ple.ple_grad_prepare(p.plan, p.rows.view(-1), p.ws)
+        if e is not None:
+            e[1].record(stream)
+        p.ple.ple_grad_apply(p.plan, N, p.grad, p.table_grad, p.ws)
+        if e is not None:
+            e[2].record(stream)
+    torch.cuda.synchronize()
+    status = p.ple.ple_status(p.table_grad.device)
+    if status != p.ple.PLE_OK:
+        raise SystemExit(f"libple async status {status}")
+    prep = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    app = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    gbs = p.bwd_bytes() / (app * 1e-3) / 1e9
+    return {"prepare_ms": prep, "apply_ms": app, "apply_gb_per_s": gbs, "apply_frac_of_measured": gbs / peak,
+            "apply_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+            "what": "ple_grad_prepare (sort) and ple_grad_apply (fold) timed apart, CUDA events, L2 flushed "
+                    "before each prepare, outside the timed steps"}
+
+
 def size_matched_copy_gbs(nbytes: int, flush_l2, stream, device, reps: int = 10) -> float:
     """GB/s of a plain device-to-device copy moving the same bytes (nbytes/2
     read, nbytes/2 written): the practical ceiling for a kernel of this size,
@@ -552,7 +587,8 @@ def main():
                     "workload": bwd_part.w.name,
                     "traffic": traffic_from_profiles(f"grad_scatter_{bwd_part.w.name}", GRAD_SRC),
                     "kernel": "ple_grad_scatter (sort + fold kernels)", "unique_rows": bwd_part.U,
-                    "peak_source": f"{peak_kind} hbm_gbs"}
+                    "peak_source": f"{peak_kind} hbm_gbs",
+                    "split": backward_split(bwd_part, flush_l2, stream, peak)}
         if bwd_part.ms_bwd > fwd_part.ms_fwd:
             roofline = bwd_roof
 
